@@ -1,0 +1,440 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each ``pin_*`` takes the oracle module as an argument, so the same pins can
+be run against deliberately broken copies of it (``test_oracle_pins.py``
+plants such mistakes on the CPU and checks that some pin catches each one).
+
+Sources of truth used here:
+* a hand-worked example (``golden/q0_worked_example.json``),
+* closed forms: with K >= #history and equal scores the method is dense
+  causal attention with history logits shifted by -ln(#history); with K = 0
+  it is block-diagonal causal attention (SAS review (paper.oopus.info),
+  §2.3 eq. o_SAS and §2.4 eq. log g),
+* library routines: torch's scaled_dot_product_attention (fp64, CPU) with an
+  additive mask, scipy's logsumexp,
+* the rank definition of Top-K with the lower-index tie-break,
+* brute force with Python loops on tiny inputs,
+* central finite differences in fp64,
+* invariants: shift invariance in s, exact zero influence of unselected K/V,
+  rows of ds sum to zero, probabilities sum to one.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+from scipy.special import logsumexp as sp_logsumexp
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+BLOCK = 64
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _sdpa(q_rows, keys, vals, bias, scale):
+    """torch SDPA in fp64 on one head: q_rows [T,D], keys/vals [U,D], bias [T,U]."""
+    q_t = torch.from_numpy(np.ascontiguousarray(q_rows))[None, None]
+    k_t = torch.from_numpy(np.ascontiguousarray(keys))[None, None]
+    v_t = torch.from_numpy(np.ascontiguousarray(vals))[None, None]
+    m_t = torch.from_numpy(np.ascontiguousarray(bias))[None, None]
+    return F.scaled_dot_product_attention(q_t, k_t, v_t, attn_mask=m_t, scale=scale)[0, 0].numpy()
+
+
+def _rank_select(row, K):
+    """Top-K by the rank definition: j is kept iff #{better} < K, where m beats
+    j when s_m > s_j, or s_m == s_j and m < j."""
+    n = len(row)
+    out = []
+    for j in range(n):
+        rank = sum(1 for m in range(n) if row[m] > row[j]) + sum(1 for m in range(j) if row[m] == row[j])
+        if rank < K:
+            out.append(j)
+    return out
+
+
+# ---------------------------------------------------------------------------
+def pin_topk_rank(O):
+    r = np.random.default_rng(11)
+    for trial in range(400):
+        nh = int(r.integers(0, 48))
+        K = int(r.integers(0, 14))
+        if trial % 3 == 0:
+            row = r.choice(np.array([-1.5, -0.0, 0.0, 0.25, 2.0, 3.0]), size=nh)
+        elif trial % 3 == 1:
+            row = np.full(nh, 0.625)
+        else:
+            row = r.standard_normal(nh).astype(np.float32).astype(np.float64)
+        assert O.topk_history(row, nh, K) == _rank_select(list(row), K), (trial, row, K)
+
+
+def pin_select_gates(O):
+    s = _rand((2, 3, 11, 11), 12).astype(np.float32)
+    K = 4
+    idx, cnt, lg, lse_s = O.select(s, K, O.prefill_history(11))
+    for b in range(2):
+        for h in range(3):
+            for i in range(11):
+                row = s[b, h, i, :i].astype(np.float64)
+                assert cnt[b, h, i] == min(K, i)
+                sel = _rank_select(list(row), K)
+                assert list(idx[b, h, i, :cnt[b, h, i]]) == sel
+                assert np.all(idx[b, h, i, cnt[b, h, i]:] == -1)
+                assert np.all(np.isneginf(lg[b, h, i, cnt[b, h, i]:]))
+                if i == 0:
+                    assert np.isneginf(lse_s[b, h, i])
+                    continue
+                ref = sp_logsumexp(row)
+                assert abs(lse_s[b, h, i] - ref) <= 1e-13 * max(1.0, abs(ref))
+                gates = lg[b, h, i, :cnt[b, h, i]]
+                assert np.allclose(gates, row[sel] - ref, rtol=0, atol=1e-13)
+                assert np.all(gates <= 1e-15)
+                tot = sp_logsumexp(gates)
+                if K >= i:
+                    assert abs(tot) <= 1e-13
+                else:
+                    assert tot < -1e-9
+
+
+def pin_golden(O):
+    with open(os.path.join(HERE, "golden", "q0_worked_example.json")) as f:
+        ex = json.load(f)
+    inp, exp = ex["inputs"], ex["expect"]
+    S, D, K, sc = inp["S"], inp["D"], inp["K"], inp["sm_scale"]
+    q = np.zeros((1, S, 1, D))
+    k = np.ones((1, S, 1, D))
+    v = np.stack([np.arange(S, dtype=np.float64), np.ones(S)], axis=1)[None, :, None, :]
+    s = np.array(inp["s"], dtype=np.float64)[None, None]
+    idx, cnt, lg, lse_s = O.select(s, K, O.prefill_history(3))
+    assert idx[0, 0].tolist() == exp["idx"] and cnt[0, 0].tolist() == exp["cnt"]
+    for i in range(3):
+        e = exp["log_gate"][i][0]
+        assert np.isneginf(lg[0, 0, i, 0]) if e is None else abs(lg[0, 0, i, 0] - e) < 1e-14
+        e = exp["lse_s"][i]
+        assert np.isneginf(lse_s[0, 0, i]) if e is None else abs(lse_s[0, 0, i] - e) < 1e-14
+    o, lse = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    assert np.allclose(o[0, :, 0, 1], exp["o1_all_rows"], rtol=0, atol=1e-12)
+    for row in exp["rows"]:
+        t = row["t"]
+        assert abs(o[0, t, 0, 0] - row["o0_num"] / row["o0_den"]) < 1e-11, (t, o[0, t, 0, 0])
+        assert abs(lse[0, 0, t] - math.log(row["lse_arg"])) < 1e-12, t
+
+
+def _dense_case(seed, S=320, Hq=4, Hkv=2, D=8):
+    q = _rand((1, S, Hq, D), seed)
+    k = _rand((1, S, Hkv, D), seed + 1)
+    v = _rand((1, S, Hkv, D), seed + 2)
+    return q, k, v
+
+
+def pin_dense_equivalence(O):
+    """K >= #history and equal scores: dense causal attention, history shifted by -ln(i)."""
+    q, k, v = _dense_case(21)
+    S, Hq, D = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    NQB = S // BLOCK
+    s = np.full((1, k.shape[2], NQB, NQB), 0.7)
+    idx, cnt, lg, _ = O.select(s, NQB, O.prefill_history(NQB))
+    sc = 1.0 / math.sqrt(D)
+    o, _ = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    t = np.arange(S)[:, None]
+    u = np.arange(S)[None, :]
+    blk = t // BLOCK
+    bias = np.where(u <= t, 0.0, -np.inf)
+    hist = u < blk * BLOCK
+    bias = np.where(hist, -np.log(np.maximum(blk, 1)), bias)
+    for hq in range(Hq):
+        ref = _sdpa(q[0, :, hq], k[0, :, hq // G], v[0, :, hq // G], bias, sc)
+        assert np.allclose(o[0, :, hq], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_block_diagonal(O):
+    """K = 0: every query attends only the causal part of its own block."""
+    q, k, v = _dense_case(31)
+    S, Hq, D = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    NQB = S // BLOCK
+    s = _rand((1, k.shape[2], NQB, NQB), 32)
+    idx, cnt, lg, _ = O.select(s, 0, O.prefill_history(NQB))
+    sc = 0.3
+    o, _ = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    t = np.arange(S)[:, None]
+    u = np.arange(S)[None, :]
+    bias = np.where((u <= t) & (u // BLOCK == t // BLOCK), 0.0, -np.inf)
+    for hq in range(Hq):
+        ref = _sdpa(q[0, :, hq], k[0, :, hq // G], v[0, :, hq // G], bias, sc)
+        assert np.allclose(o[0, :, hq], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_general_sdpa(O):
+    """General Top-K: SDPA with a mask built from the rank selection and scipy gates."""
+    q, k, v = _dense_case(41, S=448, Hq=6, Hkv=2, D=8)
+    S, Hq, Hkv, D = q.shape[1], q.shape[2], k.shape[2], q.shape[3]
+    G = Hq // Hkv
+    NQB = S // BLOCK
+    s = _rand((1, Hkv, NQB, NQB), 42, 2.0).astype(np.float32)
+    K = 3
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(NQB))
+    sc = 1.0 / math.sqrt(D)
+    o, lse = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    for h in range(Hkv):
+        bias = np.full((S, S), -np.inf)
+        for i in range(NQB):
+            row = s[0, h, i, :i].astype(np.float64)
+            ls = sp_logsumexp(row) if i else 0.0
+            for j in _rank_select(list(row), K):
+                bias[i * BLOCK:(i + 1) * BLOCK, j * BLOCK:(j + 1) * BLOCK] = row[j] - ls
+            for r in range(BLOCK):
+                bias[i * BLOCK + r, i * BLOCK:i * BLOCK + r + 1] = 0.0
+        for g in range(G):
+            hq = h * G + g
+            ref = _sdpa(q[0, :, hq], k[0, :, h], v[0, :, h], bias, sc)
+            assert np.allclose(o[0, :, hq], ref, rtol=1e-12, atol=1e-12)
+            ref_lse = torch.logsumexp(torch.from_numpy(sc * q[0, :, hq] @ k[0, :, h].T + bias), dim=1).numpy()
+            assert np.allclose(lse[0, hq], ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def pin_bruteforce_loops(O):
+    """Python loops with math.exp on a tiny case, selection and gates included."""
+    S, Hq, Hkv, D, K = 192, 2, 1, 3, 1
+    q, k, v = _rand((1, S, Hq, D), 51), _rand((1, S, Hkv, D), 52), _rand((1, S, Hkv, D), 53)
+    s = _rand((1, Hkv, 3, 3), 54)
+    sc = 0.41
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(3))
+    o, lse = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    for hq in range(Hq):
+        for t in range(S):
+            i = t // BLOCK
+            hist = [float(s[0, 0, i, j]) for j in range(i)]
+            keep = {}
+            if hist:
+                best = max(range(i), key=lambda j: (hist[j], -j))
+                mx = max(hist)
+                lsum = mx + math.log(sum(math.exp(x - mx) for x in hist))
+                keep[best] = hist[best] - lsum
+            logits, rows = [], []
+            for u in range(S):
+                j = u // BLOCK
+                if j == i and u <= t:
+                    bias = 0.0
+                elif j in keep:
+                    bias = keep[j]
+                else:
+                    continue
+                dot = sum(q[0, t, hq, d] * k[0, u, 0, d] for d in range(D))
+                logits.append(sc * dot + bias)
+                rows.append(u)
+            mx = max(logits)
+            w = [math.exp(x - mx) for x in logits]
+            z = sum(w)
+            for d in range(D):
+                ref = sum(wi * v[0, u, 0, d] for wi, u in zip(w, rows)) / z
+                assert abs(o[0, t, hq, d] - ref) < 1e-12
+            assert abs(lse[0, hq, t] - (mx + math.log(z))) < 1e-12
+
+
+def _fd_case():
+    S, Hq, Hkv, D, K = 256, 2, 1, 16, 2
+    q, k, v = _rand((1, S, Hq, D), 61), _rand((1, S, Hkv, D), 62), _rand((1, S, Hkv, D), 63)
+    do = _rand((1, S, Hq, D), 64)
+    s = _rand((1, Hkv, 4, 4), 65)
+    return q, k, v, do, s, K, 0.25
+
+
+def _loss(O, q, k, v, s, do, K, sc):
+    NQB = q.shape[1] // BLOCK
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(NQB))
+    o, _ = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    return float(np.sum(o * do))
+
+
+def pin_finite_differences(O):
+    q, k, v, do, s, K, sc = _fd_case()
+    NQB = 4
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(NQB))
+    dq, dk, dv, ds, _ = O.attn_bwd(q, k, v, do, idx, cnt, lg, s, sc)
+    h = 1e-6
+    r = np.random.default_rng(66)
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(12):
+            pos = tuple(int(r.integers(0, n)) for n in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[pos] += h
+            minus[pos] -= h
+            args = dict(q=q, k=k, v=v)
+            args[name] = plus
+            lp = _loss(O, args["q"], args["k"], args["v"], s, do, K, sc)
+            args[name] = minus
+            lm = _loss(O, args["q"], args["k"], args["v"], s, do, K, sc)
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[pos]) <= 1e-6 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
+    for i in range(1, NQB):
+        row = np.sort(s[0, 0, i, :i])
+        for j in range(i):
+            assert np.all(np.abs(np.diff(row)) > 4 * h) if i > 1 else True
+            plus, minus = s.copy(), s.copy()
+            plus[0, 0, i, j] += h
+            minus[0, 0, i, j] -= h
+            fd = (_loss(O, q, k, v, plus, do, K, sc) - _loss(O, q, k, v, minus, do, K, sc)) / (2 * h)
+            assert abs(fd - ds[0, 0, i, j]) <= 1e-6 * max(1.0, abs(fd)), (i, j, fd, ds[0, 0, i, j])
+    assert np.all(ds[0, 0][np.triu_indices(NQB)] == 0.0)
+
+
+def pin_shift_invariance(O):
+    q, k, v, do, s, K, sc = _fd_case()
+    NQB = 4
+    a = O.select(s, K, O.prefill_history(NQB))
+    b = O.select(s + 3.0, K, O.prefill_history(NQB))
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    fin = np.isfinite(a[2])
+    assert np.array_equal(fin, np.isfinite(b[2]))
+    assert np.allclose(a[2][fin], b[2][fin], rtol=0, atol=1e-13)
+    oa, _ = O.attn_fwd(q, k, v, *a[:3], sc)
+    ob, _ = O.attn_fwd(q, k, v, *b[:3], sc)
+    assert np.allclose(oa, ob, rtol=0, atol=1e-12)
+    ga = O.attn_bwd(q, k, v, do, *a[:3], s, sc)
+    gb = O.attn_bwd(q, k, v, do, *b[:3], s + 3.0, sc)
+    for x, y in zip(ga[:4], gb[:4]):
+        assert np.allclose(x, y, rtol=0, atol=1e-11)
+
+
+def pin_sparsity(O):
+    """K/V outside a row's selected blocks and current block have no influence."""
+    S, Hq, Hkv, D, K = 512, 2, 1, 8, 2
+    q, k, v = _rand((1, S, Hq, D), 71), _rand((1, S, Hkv, D), 72), _rand((1, S, Hkv, D), 73)
+    do = _rand((1, S, Hq, D), 74)
+    s = _rand((1, Hkv, 8, 8), 75)
+    NQB = 8
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(NQB))
+    sc = 0.35
+    o, lse = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    for i in range(NQB):
+        keep = set(int(j) for j in idx[0, 0, i, :cnt[0, 0, i]]) | {i}
+        k2, v2 = k.copy(), v.copy()
+        for j in range(NQB):
+            if j not in keep:
+                k2[0, j * BLOCK:(j + 1) * BLOCK] = _rand((BLOCK, Hkv, D), 100 + j, 5.0)
+                v2[0, j * BLOCK:(j + 1) * BLOCK] = _rand((BLOCK, Hkv, D), 200 + j, 5.0)
+        o2, lse2 = O.attn_fwd(q, k2, v2, idx, cnt, lg, sc)
+        rs = slice(i * BLOCK, (i + 1) * BLOCK)
+        assert np.array_equal(o[0, rs], o2[0, rs]) and np.array_equal(lse[0, :, rs], lse2[0, :, rs])
+    _, dk, dv, ds, gsum = O.attn_bwd(q, k, v, do, idx, cnt, lg, s, sc)
+    picked = set(int(j) for j in idx[0, 0][idx[0, 0] >= 0])
+    never = [j for j in range(NQB - 1) if j not in picked]
+    assert never, "case should leave some key block unselected"
+    for j in never:
+        # block j is still attended by its own (diagonal) rows; zero it out of
+        # the picture by checking that only the diagonal stripe contributes
+        diag_only = O.attn_bwd(q, k, v, do, idx, cnt, lg, s, sc,
+                               stripes=[(0, hq, j) for hq in range(Hq)])
+        rs = slice(j * BLOCK, (j + 1) * BLOCK)
+        assert np.array_equal(dk[0, rs], diag_only[1][0, rs])
+        assert np.array_equal(dv[0, rs], diag_only[2][0, rs])
+    for i in range(NQB):
+        sel = set(int(j) for j in idx[0, 0, i, :cnt[0, 0, i]])
+        for j in range(i):
+            if j not in sel:
+                assert gsum[0, 0, i, j] == 0.0
+        assert abs(ds[0, 0, i].sum()) <= 1e-12 * max(1.0, np.abs(ds[0, 0, i]).sum())
+
+
+def pin_probabilities(O):
+    q, k, v = _dense_case(81)
+    NQB = q.shape[1] // BLOCK
+    s = _rand((1, 2, NQB, NQB), 82)
+    idx, cnt, lg, _ = O.select(s, 2, O.prefill_history(NQB))
+    q64, k64, v64 = q, k, v
+    for hq in range(q.shape[2]):
+        for i in range(NQB):
+            _, _, P, _ = O.fwd_stripe(q64, k64, v64, idx, cnt, lg, 0.3, 0, hq, i)
+            assert np.allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+            assert np.all(P >= 0)
+
+
+def _paged(kc_rows, vc_rows, n_pages_total, perm_seed):
+    """Scatter contiguous [L,Hkv,D] K/V rows of one sequence into 64-token pages."""
+    L, Hkv, D = kc_rows.shape
+    npg = (L + BLOCK - 1) // BLOCK
+    perm = np.random.default_rng(perm_seed).permutation(n_pages_total)[:npg]
+    kc = _rand((n_pages_total, Hkv, BLOCK, D), perm_seed + 1)
+    vc = _rand((n_pages_total, Hkv, BLOCK, D), perm_seed + 2)
+    for p in range(npg):
+        rows = slice(p * BLOCK, min(L, (p + 1) * BLOCK))
+        n = rows.stop - rows.start
+        kc[perm[p], :, :n] = kc_rows[rows].transpose(1, 0, 2)
+        vc[perm[p], :, :n] = vc_rows[rows].transpose(1, 0, 2)
+    return kc, vc, perm
+
+
+def pin_decode_vs_sdpa(O):
+    Hq, Hkv, D, K = 4, 2, 8, 3
+    G = Hq // Hkv
+    lens = [1, 64, 65, 200, 640, 700]
+    N = len(lens)
+    maxp = max((L + 63) // 64 for L in lens)
+    q = _rand((N, Hq, D), 91)
+    s = _rand((N, Hkv, 16), 92).astype(np.float32)
+    kv_len = np.array(lens)
+    kcs, vcs, pts, conts = [], [], np.zeros((N, maxp), dtype=np.int64), []
+    total = 0
+    for n, L in enumerate(lens):
+        kr, vr = _rand((L, Hkv, D), 300 + n), _rand((L, Hkv, D), 400 + n)
+        kc, vc, perm = _paged(kr, vr, 12, 500 + n)
+        kcs.append(kc)
+        vcs.append(vc)
+        pts[n, :len(perm)] = perm + total
+        total += 12
+        conts.append((kr, vr))
+    kc, vc = np.concatenate(kcs), np.concatenate(vcs)
+    idx, cnt, lg, lse_s = O.select(s[:, :, None, :], K, O.decode_history(kv_len)[:, None])
+    idx, cnt, lg = idx[:, :, 0], cnt[:, :, 0], lg[:, :, 0]
+    sc = 1.0 / math.sqrt(D)
+    o, lse = O.decode(q, kc, vc, pts, kv_len, idx, cnt, lg, sc)
+    for n, L in enumerate(lens):
+        kr, vr = conts[n]
+        c = (L - 1) // BLOCK
+        for h in range(Hkv):
+            row = s[n, h, :c].astype(np.float64)
+            bias = np.full((1, L), -np.inf)
+            bias[0, c * BLOCK:L] = 0.0
+            if c:
+                ls = sp_logsumexp(row)
+                for j in _rank_select(list(row), K):
+                    bias[0, j * BLOCK:(j + 1) * BLOCK] = row[j] - ls
+            for g in range(G):
+                hq = h * G + g
+                ref = _sdpa(q[n, hq][None], kr[:, h], vr[:, h], bias, sc)[0]
+                assert np.allclose(o[n, hq], ref, rtol=1e-12, atol=1e-12), (n, hq)
+
+
+def pin_decode_vs_prefill(O):
+    """The last row of a full prefill block equals a decode query at that position."""
+    S, Hq, Hkv, D, K = 512, 4, 2, 8, 2
+    G = Hq // Hkv
+    q, k, v = _rand((1, S, Hq, D), 111), _rand((1, S, Hkv, D), 112), _rand((1, S, Hkv, D), 113)
+    NQB = S // BLOCK
+    s = _rand((1, Hkv, NQB, NQB), 114)
+    sc = 0.3
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(NQB))
+    o, lse = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    kc, vc, perm = _paged(k[0], v[0], 20, 115)
+    pt = perm[None]
+    kv_len = np.array([S])
+    sd = s[:, :, NQB - 1, :].copy()
+    didx, dcnt, dlg, _ = O.select(sd[:, :, None, :], K, O.decode_history(kv_len)[:, None])
+    od, lsed = O.decode(q[:, S - 1], kc, vc, pt, kv_len, didx[:, :, 0], dcnt[:, :, 0], dlg[:, :, 0], sc)
+    assert np.allclose(od[0], o[0, S - 1], rtol=1e-12, atol=1e-12)
+    assert np.allclose(lsed[0], lse[0, :, S - 1], rtol=1e-12, atol=1e-12)
+    assert G == 2
+
+
+ALL_PINS = [
+    pin_topk_rank, pin_select_gates, pin_golden, pin_dense_equivalence, pin_block_diagonal,
+    pin_general_sdpa, pin_bruteforce_loops, pin_finite_differences, pin_shift_invariance,
+    pin_sparsity, pin_probabilities, pin_decode_vs_sdpa, pin_decode_vs_prefill,
+]

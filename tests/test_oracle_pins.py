@@ -1,0 +1,61 @@
+"""The oracle against its pins, and the pins against planted oracle mistakes.
+
+Every mutant below is a plausible slip in ``oracle/sas_oracle.py`` (a dropped
+term, a wrong sign, index or operand, a misplaced scale). Each is planted in
+a copy of the oracle's source on the CPU, and at least one pin must fail on
+it; otherwise the pins would not be able to tell a wrong oracle from a right
+one.
+"""
+import importlib.util
+import inspect
+import types
+
+import pytest
+
+from oracle import sas_oracle
+from tests import oracle_pins as pins
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(pin):
+    pin(sas_oracle)
+
+
+MUTANTS = {
+    "lse_over_selected_only": ("lse = logsumexp(row)\n", "lse = logsumexp(row[sel])\n"),
+    "gate_sign_flipped": ("log_gate[b, h, r, slot] = row[j] - lse", "log_gate[b, h, r, slot] = lse - row[j]"),
+    "tie_break_higher_index": ("np.lexsort((np.arange(nh), -s_row))", "np.lexsort((-np.arange(nh), -s_row))"),
+    "causal_mask_off_by_one": ("np.where(u <= t, 0.0, NEG_INF)", "np.where(u < t + (t == 0), 0.0, NEG_INF)"),
+    "current_block_gated": ("bias[:, i * BLOCK:(i + 1) * BLOCK] = np.where(u <= t, 0.0, NEG_INF)",
+                            "bias[:, i * BLOCK:(i + 1) * BLOCK] = np.where(u <= t, (gates[0] if gates else 0.0), NEG_INF)"),
+    "scale_applied_to_gate": ("L = sm_scale * (Qi @ Kh.T) + stripe_bias(i, S, sel, gates)",
+                              "L = sm_scale * ((Qi @ Kh.T) + stripe_bias(i, S, sel, gates))"),
+    "gqa_head_map_modulo": ("h = hq // G\n    sel, gates", "h = hq % k.shape[2]\n    sel, gates"),
+    "jacobian_term_dropped": ("ds[b, h, i, :i] = -p * tot", "ds[b, h, i, :i] = 0.0 * p * tot"),
+    "dk_missing_scale": ("dk[b, :, h, :] += sm_scale * (dS.T @ Qi)", "dk[b, :, h, :] += (dS.T @ Qi)"),
+    "dP_wrong_operand": ("dP = dOi @ Vh.T", "dP = dOi @ Kh.T"),
+    "gate_sum_wrong_axis": ("reshape(BLOCK, i, BLOCK).sum(axis=(0, 2))", "reshape(BLOCK, i, BLOCK).sum(axis=(2, 0))[::-1]"),
+    "Dr_dropped": ("dS = P * (dP - Dr)", "dS = P * dP"),
+    "decode_current_block_short": ("bias[c * BLOCK:L] = 0.0", "bias[c * BLOCK:L - 1 + (L - 1 == c * BLOCK)] = 0.0"),
+    "decode_history_includes_current": ("return (_i64(kv_len) - 1) // BLOCK", "return (_i64(kv_len) + BLOCK - 1) // BLOCK"),
+}
+
+
+def _mutant(src_from, src_to):
+    src = inspect.getsource(sas_oracle)
+    assert src.count(src_from) == 1, src_from
+    mod = types.ModuleType("sas_oracle_mutant")
+    exec(compile(src.replace(src_from, src_to), "sas_oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    mod = _mutant(*MUTANTS[name])
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(mod)
+        except Exception:          # an assertion, or a crash the slip causes
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name!r}"

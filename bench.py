@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the SAS gated block-sparse attention hot path on B200.
+
+One step = the whole path on one batch of seeded synthetic input:
+  prefill/training part on the Qwen3-8B-shaped 32k layer (B=1, S=32768,
+  32/8 heads, D=128, K=32): select -> forward -> backward (dq, dk, dv, ds);
+  decode part on 64 paged sequences (8k..64k context, 32/8 heads, K=32):
+  select -> paged decode.
+`value` is the prefill part's throughput in TFLOPS counting only attended
+64x64 tiles (14*64*64*D flops per tile: 4 forward, 10 backward) over the
+device time of select+forward+backward. Decode is reported beside it in GB/s
+of algorithmic HBM bytes and tokens/s.
+
+Multi-GPU (torchrun): every rank runs its own independent replica of the
+workload (different seed), no collective in the data path; the timed region
+is bracketed by barriers and the max over ranks is reported (weak scaling).
+
+`--impl reference` times the fp64 CPU oracle instead (rank 0 only), each
+step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+BLOCK = 64
+L2_BYTES = 126 * 2**20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill", default="qwen3-8b-32k")
+    ap.add_argument("--decode", default="decode-64seq")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return dict(hbm=float(m["hbm_gbs"]), bf16=float(m["bf16_tflops"]),
+                    bf16_sustained=float(m.get("bf16_tflops_sustained", m["bf16_tflops"])), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# work counts (algorithmic)
+# ---------------------------------------------------------------------------
+
+def prefill_tiles(cfg):
+    """Attended 64x64 tiles over all query heads: sum over query blocks of (min(K, i) + 1)."""
+    per_head = sum(min(cfg.K, i) + 1 for i in range(cfg.NQB))
+    return per_head * cfg.B * cfg.Hq
+
+
+def decode_bytes(cfg, kv_len, cnt):
+    """Algorithmic HBM bytes of one decode call: kept K/V pages (full history
+    pages, the current block's valid tokens), q, o, selection and page ids."""
+    import torch
+    kv_len = kv_len.to(torch.int64).cpu()
+    cnt = cnt.to(torch.int64).cpu()                       # [N, Hkv]
+    c = (kv_len - 1) // BLOCK
+    cur_tokens = (kv_len - c * BLOCK)[:, None]             # [N, 1]
+    tokens = cnt * BLOCK + cur_tokens                      # [N, Hkv]
+    kv = int(tokens.sum()) * cfg.D * 2 * 2
+    qo = cfg.N * cfg.Hq * cfg.D * 2 * 2
+    sel = cfg.N * cfg.Hkv * (cfg.K * 8 + 4) + int((cnt + 1).sum()) * 4 + cfg.N * 4
+    return kv + qo + sel
+
+
+def select_bytes(nh_total, rows, K):
+    return nh_total * 4 + rows * (K * 8 + 8)
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
+                   "--format=csv,noheader,nounits", "-lms", "100"]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["clock sampling unavailable"], samples=0)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
+                    reasons=sorted(reasons), samples=len(sm))
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+
+    from trainable_gated_block_b200 import build, inputs, sas
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=torch.device("cuda", local))
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    sas.lib()
+    dev = torch.device("cuda", local)
+    peaks = _peaks()
+
+    pc = inputs.workload(a.prefill)
+    dc = inputs.workload(a.decode)
+    px = inputs.make_prefill(pc, seed=pc.seed + 1000 * rank)
+    dx = inputs.make_decode(dc, seed=dc.seed + 1000 * rank)
+    P = {k: v.to(dev) for k, v in px.items()}
+    Dd = {k: v.to(dev) for k, v in dx.items()}
+    sc_p = 1.0 / math.sqrt(pc.D)
+    ws_b = torch.empty(sas.bwd_workspace_bytes(P["q"], P["k"], pc.K), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(sas.decode_workspace_bytes(dc.N, dc.Hq, dc.Hkv, dc.D, dc.K), dtype=torch.uint8, device=dev)
+
+    names = ["select", "fwd", "bwd", "dselect", "decode"]
+
+    def step(rec):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)] if rec else None
+        if rec:
+            ev[0].record()
+        sel = sas.select(P["s"], pc.K)
+        if rec:
+            ev[1].record()
+        o, lse = sas.attn_fwd(P["q"], P["k"], P["v"], sel[0], sel[1], sel[2], sc_p)
+        if rec:
+            ev[2].record()
+        grads = sas.attn_bwd(P["q"], P["k"], P["v"], o, P["do"], lse, P["s"], sel[3], sel[0], sel[1], sel[2],
+                             sc_p, workspace=ws_b)
+        if rec:
+            ev[3].record()
+        dsel = sas.select(Dd["s"], dc.K, kv_len=Dd["kv_len"])
+        if rec:
+            ev[4].record()
+        od, _ = sas.decode_paged(Dd["q"], Dd["k_cache"], Dd["v_cache"], Dd["page_table"], Dd["kv_len"],
+                                 dsel[0], dsel[1], dsel[2], workspace=ws_d, with_lse=False)
+        if rec:
+            ev[5].record()
+        return ev, (o, grads, od, dsel)
+
+    for _ in range(a.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    sas.get_error_flag()
+    _, (_, _, _, dsel) = step(False)
+    dec_bytes = decode_bytes(dc, dx["kv_len"], dsel[1])
+    torch.cuda.synchronize()
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = sas.kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    evs = [step(True)[0] for _ in range(a.steps)]
+    t1.record()
+    torch.cuda.synchronize()
+    launches = sas.kernel_launches() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    sas.get_error_flag()
+    total_ms = t0.elapsed_time(t1)
+    part_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / a.steps for i, n in enumerate(names)}
+    prefill_ms = part_ms["select"] + part_ms["fwd"] + part_ms["bwd"]
+    dec_ms = part_ms["dselect"] + part_ms["decode"]
+    if world > 1:
+        t = torch.tensor([total_ms, prefill_ms, dec_ms] + [part_ms[n] for n in names], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, prefill_ms, dec_ms = float(t[0]), float(t[1]), float(t[2])
+        part_ms = {n: float(t[3 + i]) for i, n in enumerate(names)}
+
+    tiles = prefill_tiles(pc)
+    unit_flops = 64 * 64 * pc.D
+    flops_fb = 14 * unit_flops * tiles
+    tflops = world * flops_fb / (prefill_ms * 1e-3) / 1e12
+    bwd_tf = 10 * unit_flops * tiles / (part_ms["bwd"] * 1e-3) / 1e12
+    fwd_tf = 4 * unit_flops * tiles / (part_ms["fwd"] * 1e-3) / 1e12
+    dec_gbs = dec_bytes / (part_ms["decode"] * 1e-3) / 1e9
+    nh_pre = sum(range(pc.NQB)) * pc.B * pc.Hkv
+    sel_bytes = select_bytes(nh_pre, pc.B * pc.Hkv * pc.NQB, pc.K)
+    sel_gbs = sel_bytes / (part_ms["select"] * 1e-3) / 1e9
+    tag = "of measured" if peaks["source"] == "measured" else "of fallback"
+    kernels = {
+        "select": dict(bound="hbm", achieved=sel_gbs, peak=peaks["hbm"], unit="GB/s", frac=sel_gbs / peaks["hbm"],
+                       ms=part_ms["select"], bytes=sel_bytes),
+        "fwd": dict(bound="tensor", achieved=fwd_tf, peak=peaks["bf16_sustained"], unit="TFLOP/s",
+                    frac=fwd_tf / peaks["bf16_sustained"], ms=part_ms["fwd"]),
+        "bwd": dict(bound="tensor", achieved=bwd_tf, peak=peaks["bf16_sustained"], unit="TFLOP/s",
+                    frac=bwd_tf / peaks["bf16_sustained"], ms=part_ms["bwd"]),
+        "decode": dict(bound="hbm", achieved=dec_gbs, peak=peaks["hbm"], unit="GB/s", frac=dec_gbs / peaks["hbm"],
+                       ms=part_ms["decode"], bytes=dec_bytes, tokens_per_s=dc.N / (part_ms["decode"] * 1e-3)),
+    }
+    dom = max(("fwd", "bwd", "decode", "select"), key=lambda n: part_ms[n])
+    kd = kernels[dom]
+    roofline = dict(bound=kd["bound"], achieved=round(kd["achieved"], 3), peak=kd["peak"], unit=kd["unit"],
+                    frac=round(kd["frac"], 4), traffic=None, kernel=f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}",
+                    peak_note=f"{tag} ({'sustained bf16' if kd['bound'] == 'tensor' else 'HBM copy'})")
+
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, world, dist, dev)
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": "SAS gated block-sparse attn fwd+bwd TFLOPS & decode HBM GB/s vs roofline",
+            "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v/dO, pooled stand-in scores)",
+            "config": {
+                "workload": f"{pc.name} select+fwd+bwd, then {dc.name} select+paged decode",
+                "prefill": dict(B=pc.B, S=pc.S, Hq=pc.Hq, Hkv=pc.Hkv, D=pc.D, K=pc.K, block=BLOCK,
+                                attended_tiles=tiles, flops_per_step=flops_fb),
+                "decode": dict(N=dc.N, Hq=dc.Hq, Hkv=dc.Hkv, D=dc.D, K=dc.K, ctx="8k..64k",
+                               algorithmic_bytes=dec_bytes),
+                "l2": "inputs larger than L2 (prefill q/k/v/o/dO about 0.9 GB, decode pages 0.54 GB per step)",
+                "parallelism": f"replicas x{world} (no collective)",
+            },
+            "decode": dict(gbs=round(dec_gbs, 1), tokens_per_s=round(world * dc.N / (dec_ms * 1e-3), 1),
+                           us_decode_kernel=round(part_ms["decode"] * 1e3, 2), us_select=round(part_ms["dselect"] * 1e3, 2),
+                           frac_hbm=round(dec_gbs / peaks["hbm"], 4)),
+            "part_ms": {k: round(v, 4) for k, v in part_ms.items()},
+            "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                        for k, v in kernels.items()},
+            "roofline": roofline,
+            "clocks": clk,
+            "gpu_launches": launches,
+            "e2e": e2e,
+        }
+        if world == 1 and not a.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(pc, px, a.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line))
+
+
+def run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, world, dist, dev):
+    """Same step through the public API, inputs copied from pinned host memory
+    every step and every result read back to pinned host memory."""
+    hin_p = {k: px[k].pin_memory() for k in ("q", "k", "v", "do", "s")}
+    hin_d = {k: dx[k].pin_memory() for k in ("q", "s", "kv_len", "page_table")}
+    h2d = sum(t.numel() * t.element_size() for t in list(hin_p.values()) + list(hin_d.values()))
+    outs = {}
+
+    def step(rec):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if rec else None
+        if rec:
+            ev[0].record()
+        for k, t in hin_p.items():
+            P[k].copy_(t, non_blocking=True)
+        sel = sas.select(P["s"], pc.K)
+        o, lse = sas.attn_fwd(P["q"], P["k"], P["v"], sel[0], sel[1], sel[2], sc_p)
+        dq, dk, dv, ds = sas.attn_bwd(P["q"], P["k"], P["v"], o, P["do"], lse, P["s"], sel[3], sel[0], sel[1],
+                                      sel[2], sc_p, workspace=ws_b)
+        res = dict(o=o, dq=dq, dk=dk, dv=dv, ds=ds)
+        for k, t in res.items():
+            if k not in outs:
+                outs[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            outs[k].copy_(t, non_blocking=True)
+        if rec:
+            ev[1].record()
+        for k, t in hin_d.items():
+            Dd[k].copy_(t, non_blocking=True)
+        dsel = sas.select(Dd["s"], dc.K, kv_len=Dd["kv_len"])
+        od, _ = sas.decode_paged(Dd["q"], Dd["k_cache"], Dd["v_cache"], Dd["page_table"], Dd["kv_len"],
+                                 dsel[0], dsel[1], dsel[2], workspace=ws_d, with_lse=False)
+        if "od" not in outs:
+            outs["od"] = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
+        outs["od"].copy_(od, non_blocking=True)
+        if rec:
+            ev[2].record()
+        return ev
+
+    for _ in range(max(1, a.warmup)):
+        step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [step(True) for _ in range(a.steps)]
+    torch.cuda.synchronize()
+    sas.get_error_flag()
+    pre = sum(e[0].elapsed_time(e[1]) for e in evs) / a.steps
+    dec = sum(e[1].elapsed_time(e[2]) for e in evs) / a.steps
+    if world > 1:
+        t = torch.tensor([pre, dec], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        pre, dec = float(t[0]), float(t[1])
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    return dict(value=round(world * flops_fb / (pre * 1e-3) / 1e12, 3), unit="TFLOPS",
+                h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
+                ms_prefill=round(pre, 3), ms_decode=round(dec, 3),
+                decode_tokens_per_s=round(world * dc.N / (dec * 1e-3), 1))
+
+
+# ---------------------------------------------------------------------------
+# the fp64 CPU oracle (the cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def _oracle_stripes(pc, px, budget_s, max_stripes=10**9):
+    """Time oracle forward+backward stripes of the workload until the budget is spent."""
+    import numpy as np
+
+    from oracle import sas_oracle as O
+    # query head 0 and its KV head only (G = 1 view), so the oracle's full-size
+    # output buffers stay small
+    q, do = (O._f64(px[n][:1, :, :1]) for n in ("q", "do"))
+    k, v = (O._f64(px[n][:1, :, :1]) for n in ("k", "v"))
+    s = px["s"][:1, :1].numpy()
+    rows = [pc.NQB - 1 - 7 * r for r in range(pc.NQB // 7)]      # spread over the sequence
+    flops, n, t_spent = 0, 0, 0.0
+    sc = 1.0 / math.sqrt(pc.D)
+    for i in rows:
+        if t_spent >= budget_s or n >= max_stripes:
+            break
+        s1 = s[:1, :1, i:i + 1, :]
+        idx1, cnt1, lg1, _ = O.select(s1, pc.K, np.array([[i]]))
+        idx = np.full((1, 1, pc.NQB, pc.K), -1, dtype=np.int32)
+        cnt = np.zeros((1, 1, pc.NQB), dtype=np.int32)
+        lg = np.full((1, 1, pc.NQB, pc.K), -np.inf)
+        idx[0, 0, i], cnt[0, 0, i], lg[0, 0, i] = idx1[0, 0, 0], cnt1[0, 0, 0], lg1[0, 0, 0]
+        t0 = time.perf_counter()
+        O.attn_fwd(q, k, v, idx, cnt, lg, sc, stripes=[(0, 0, i)])
+        O.attn_bwd(q, k, v, do, idx, cnt, lg, s, sc, stripes=[(0, 0, i)])
+        t_spent += time.perf_counter() - t0
+        flops += 14 * 64 * 64 * pc.D * (int(cnt[0, 0, i]) + 1)
+        n += 1
+    return flops, n, t_spent
+
+
+def cpu_baseline(pc, px, budget_s):
+    flops, n, t = _oracle_stripes(pc, px, budget_s)
+    return dict(value=flops / t / 1e12, unit="TFLOPS", cores=_blas_threads(), kind="oracle",
+                sample=f"fp64 oracle forward+backward of {n} 64-row stripes (batch 0, head 0) of the "
+                       f"{pc.name} workload, {t:.1f} s, counted as attended-tile flops")
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from trainable_gated_block_b200 import inputs
+    pc = inputs.workload(a.prefill)
+    px = inputs.make_prefill(pc)
+    per_step = 2
+    for _ in range(a.warmup):
+        _oracle_stripes(pc, px, 0.0, max_stripes=1)
+    tot_f, tot_t, tot_n = 0, 0.0, 0
+    for _ in range(a.steps):
+        f, n, t = _oracle_stripes(pc, px, 1e9, max_stripes=per_step)
+        tot_f, tot_t, tot_n = tot_f + f, tot_t + t, tot_n + n
+    value = tot_f / tot_t / 1e12
+    cores = _blas_threads()
+    sample = (f"each step: fp64 oracle forward+backward of {per_step} 64-row stripes of the {pc.name} "
+              f"workload (attended-tile flops); {tot_n} stripes in {tot_t:.1f} s")
+    line = {
+        "impl": "reference",
+        "metric": "SAS gated block-sparse attn fwd+bwd TFLOPS & decode HBM GB/s vs roofline",
+        "value": value, "unit": "TFLOPS", "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": tot_t / a.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{pc.name} select+fwd+bwd (oracle sample)"},
+        "cpu_baseline": dict(value=value, unit="TFLOPS", cores=cores, kind="oracle", sample=sample),
+        "e2e": dict(value=value, unit="TFLOPS", h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)

@@ -1,0 +1,191 @@
+"""ctypes binding of libsas.so (C ABI in include/sas.h).
+
+Argument marshalling only: shapes are read off torch tensors, outputs and
+workspaces are allocated with torch on the input's device, and every call
+goes straight to the library on torch's current CUDA stream. There is no
+fallback: if libsas.so is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsas.so")
+
+SAS_OK, SAS_ERR_INVALID_ARG, SAS_ERR_UNSUPPORTED, SAS_ERR_CUDA, SAS_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SAS_F32, SAS_BF16 = 0, 1
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+# name -> (restype, argtypes); must match include/sas.h
+SIGNATURES = {
+    "sas_last_error": (ctypes.c_char_p, []),
+    "sas_kernel_launches": (ctypes.c_uint64, []),
+    "sas_get_error_flag": (_I, [_P]),
+    "sas_select": (_I, [_P, _I, _I, _I, _I, _P, _I, _I, _P, _P, _P, _P, _P]),
+    "sas_attn_fwd": (_I, [_I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _F, _P, _P, _P]),
+    "sas_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
+    "sas_attn_bwd": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P,
+                          _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _Z, _P]),
+    "sas_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "sas_decode_paged": (_I, [_P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                              _P, _P, _P, _F, _P, _P, _P, _Z, _P]),
+}
+
+
+class SasError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libsas status {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsas.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m trainable_gated_block_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(code: int):
+    if code != SAS_OK:
+        raise SasError(code, lib().sas_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return SAS_BF16
+    if t.dtype == torch.float32:
+        return SAS_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def kernel_launches() -> int:
+    """Kernels libsas.so has enqueued in this process so far."""
+    return int(lib().sas_kernel_launches())
+
+
+def get_error_flag(stream=None):
+    """Synchronise the stream and raise if a kernel flagged bad data or a timeout."""
+    _check(lib().sas_get_error_flag(_stream(stream)))
+
+
+def select(s, K: int, kv_len=None, block_size: int = 64):
+    """Top-K + log-gates. Prefill: s [B,Hkv,NQB,ld]. Decode: s [N,Hkv,ld], kv_len [N].
+
+    Returns idx, cnt, log_gate, lse_s shaped [B,Hkv,R,K], [B,Hkv,R], [B,Hkv,R,K],
+    [B,Hkv,R] (decode: R dimension dropped).
+    """
+    decode = kv_len is not None
+    s4 = s[:, :, None, :] if decode else s
+    _contig(s4, kv_len)
+    B, H, R, ld = s4.shape
+    dev = s.device
+    idx = torch.empty((B, H, R, K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B, H, R), dtype=torch.int32, device=dev)
+    lg = torch.empty((B, H, R, K), dtype=torch.float32, device=dev)
+    lse_s = torch.empty((B, H, R), dtype=torch.float32, device=dev)
+    _check(lib().sas_select(_ptr(s4), B, H, R, ld, _ptr(kv_len), block_size, K,
+                            _ptr(idx), _ptr(cnt), _ptr(lg), _ptr(lse_s), _stream()))
+    if decode:
+        return idx[:, :, 0], cnt[:, :, 0], lg[:, :, 0], lse_s[:, :, 0]
+    return idx, cnt, lg, lse_s
+
+
+def attn_fwd(q, k, v, idx, cnt, log_gate, sm_scale=None, block_size: int = 64):
+    """Gated block-sparse causal attention forward. Returns o [B,S,Hq,D], lse [B,Hq,S]."""
+    _contig(q, k, v, idx, cnt, log_gate)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    K = idx.shape[-1]
+    sm_scale = 1.0 / math.sqrt(D) if sm_scale is None else sm_scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _check(lib().sas_attn_fwd(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), B, S, Hq, Hkv, D, block_size, K,
+                              _ptr(idx), _ptr(cnt), _ptr(log_gate), sm_scale, _ptr(o), _ptr(lse), _stream()))
+    return o, lse
+
+
+def bwd_workspace_bytes(q, k, K: int) -> int:
+    B, S, Hq, D = q.shape
+    return int(lib().sas_attn_bwd_workspace_size(_dtype_code(q), B, S, Hq, k.shape[2], D, K))
+
+
+def attn_bwd(q, k, v, o, do, lse, s, lse_s, idx, cnt, log_gate, sm_scale=None, block_size: int = 64,
+             workspace=None):
+    """Backward. Returns dq, dk, dv (input dtype) and ds fp32 [B,Hkv,NQB,ld_s]."""
+    _contig(q, k, v, o, do, lse, s, lse_s, idx, cnt, log_gate)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    K = idx.shape[-1]
+    ld_s = s.shape[-1]
+    sm_scale = 1.0 / math.sqrt(D) if sm_scale is None else sm_scale
+    need = bwd_workspace_bytes(q, k, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ds = torch.empty(s.shape, dtype=torch.float32, device=q.device)
+    _check(lib().sas_attn_bwd(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                              _ptr(s), ld_s, _ptr(lse_s), _ptr(idx), _ptr(cnt), _ptr(log_gate),
+                              B, S, Hq, Hkv, D, block_size, K, sm_scale,
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds), _ptr(workspace), workspace.numel(),
+                              _stream()))
+    return dq, dk, dv, ds
+
+
+def decode_workspace_bytes(N: int, Hq: int, Hkv: int, D: int, K: int) -> int:
+    return int(lib().sas_decode_workspace_size(N, Hq, Hkv, D, K))
+
+
+def decode_paged(q, k_cache, v_cache, page_table, kv_len, idx, cnt, log_gate, sm_scale=None,
+                 page_size: int = 64, workspace=None, with_lse: bool = True):
+    """Paged decode. q [N,Hq,D]; caches [P,Hkv,64,D]. Returns o [N,Hq,D] and lse [N,Hq] (or None)."""
+    _contig(q, k_cache, v_cache, page_table, kv_len, idx, cnt, log_gate)
+    N, Hq, D = q.shape
+    P, Hkv = k_cache.shape[0], k_cache.shape[1]
+    K = idx.shape[-1]
+    sm_scale = 1.0 / math.sqrt(D) if sm_scale is None else sm_scale
+    need = decode_workspace_bytes(N, Hq, Hkv, D, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    _check(lib().sas_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), P, _ptr(page_table),
+                                  page_table.shape[1], _ptr(kv_len), N, Hq, Hkv, D, page_size, K,
+                                  _ptr(idx), _ptr(cnt), _ptr(log_gate), sm_scale, _ptr(o), _ptr(lse),
+                                  _ptr(workspace), workspace.numel(), _stream()))
+    return o, lse

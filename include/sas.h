@@ -179,6 +179,33 @@ sas_status sas_decode_paged(const void *q, const void *k_cache, const void *v_ca
                             const float *log_gate, float sm_scale, void *o, float *lse,
                             void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * sas_decode_paged_noalloc - sas_decode_paged for callers that cannot
+ * allocate device memory. The SAS pages have no counterpart to this call: it
+ * exists for callers such as a serving engine that gives nearly all of the
+ * GPU to its KV-cache pool at start-up, or a plain C host that holds only
+ * its input and output buffers and no device allocator.
+ *
+ * Arguments, outputs and errors are those of sas_decode_paged, without the
+ * workspace: the split-KV partials go to a 16 MiB array that the library
+ * reserves in device memory when it is loaded (every GPU that loads the
+ * library holds it until the process exits). Sizes whose partials need more
+ * than 16 MiB (sas_decode_workspace_size(N, Hq, Hkv, D, K) > 16 MiB) are
+ * rejected with SAS_ERR_INVALID_ARG before anything runs. No device memory
+ * is allocated or freed by the call.
+ * All calls on one device share that array, which keeps the last call's
+ * contents; nothing in it needs to start at zero. Calls that overlap on the
+ * GPU (on different streams, or from threads without ordering) race on it.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.
+ */
+sas_status sas_decode_paged_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                    int num_pages, const int32_t *page_table, int max_pages,
+                                    const int32_t *kv_len, int N, int Hq, int Hkv, int D,
+                                    int page_size, int K, const int32_t *idx, const int32_t *cnt,
+                                    const float *log_gate, float sm_scale, void *o, float *lse,
+                                    void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -12,6 +12,9 @@ namespace sas {
 // Process-wide count of kernels enqueued by the launchers below.
 void count_launches(int n);
 
+// Sets the message sas_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 cudaError_t launch_select(const float* s, int B, int Hkv, int n_rows, int ld_s,
                           const int32_t* kv_len, int K, int max_hist,
                           int32_t* idx, int32_t* cnt, float* log_gate, float* lse_s,

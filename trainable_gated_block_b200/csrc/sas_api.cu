@@ -73,6 +73,7 @@ sas_status check_attn_shape(sas_dtype dtype, const void* q, const void* k, const
 namespace sas {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+void set_last_error(const char* msg) { snprintf(g_msg, sizeof g_msg, "%s", msg); }
 }  // namespace sas
 
 extern "C" {

@@ -37,6 +37,8 @@ SIGNATURES = {
     "sas_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sas_decode_paged": (_I, [_P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                               _P, _P, _P, _F, _P, _P, _P, _Z, _P]),
+    "sas_decode_paged_noalloc": (_I, [_P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                      _P, _P, _P, _F, _P, _P, _P]),
 }
 
 

@@ -30,6 +30,8 @@ struct AttnArgs {
 
 // fp32 (and reference-grade generic) CUDA-core path.
 cudaError_t launch_fwd_simt(const AttnArgs& a, bool bf16, void* o, float* lse, cudaStream_t st);
+// bf16, D = 128: tcgen05 tensor-core path.
+cudaError_t launch_fwd_sm100(const AttnArgs& a, void* o, float* lse, cudaStream_t st);
 
 struct BwdArgs {
     AttnArgs a;

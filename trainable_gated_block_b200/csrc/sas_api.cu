@@ -125,7 +125,9 @@ sas_status sas_attn_fwd(sas_dtype dtype, const void* q, const void* k, const voi
     int* st = status_ptr();
     if (!st) return fail(SAS_ERR_CUDA, "sas_attn_fwd: no CUDA device");
     sas::AttnArgs a{q, k, v, B, S, Hq, Hkv, D, K, idx, cnt, log_gate, sm_scale, st};
-    cudaError_t e = sas::launch_fwd_simt(a, dtype == SAS_BF16, o, lse, static_cast<cudaStream_t>(stream));
+    cudaError_t e = (dtype == SAS_BF16 && D == 128)
+                        ? sas::launch_fwd_sm100(a, o, lse, static_cast<cudaStream_t>(stream))
+                        : sas::launch_fwd_simt(a, dtype == SAS_BF16, o, lse, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "sas_attn_fwd");
 }
 

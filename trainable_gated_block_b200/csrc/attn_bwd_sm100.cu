@@ -1,0 +1,837 @@
+// Gated block-sparse causal attention backward on the sm_100a tensor cores.
+//
+// SAS review (paper.oopus.info) §2.6: the probabilities are recomputed tile
+// by tile from the saved row LSE (never the full matrix), and the gradient
+// of a kept block's gate is the sum of the logit gradients inside the block;
+// §2.4, eq. log g: the scores receive it through the Jacobian of s - LSE(s)
+// (ds_finalize_kernel). Per attended tile of query block i and key block j:
+//   P = exp(sm_scale q.k + log g - lse),  dP = dO V^T,  dS = P (dP - Dr),
+//   dQ += sm_scale dS K,  dK += sm_scale dS^T Q,  dV += P^T dO,
+//   Gsum[i][slot(j)] += sum(dS)           (kept blocks only).
+//
+// Two tensor-core kernels, no floating-point atomics on dq/dk/dv:
+//  * dq_kernel (query-stationary, like the forward): item = (b, h, i, head
+//    group); per kept block S, dP (tcgen05, SS), dS written back to TMEM as
+//    bf16 and dQ += dS K (tcgen05, A from TMEM); dQ stays in TMEM across the
+//    item. Also the per-block gate gradients.
+//  * dkv_kernel (key-stationary): item = (b, h, j); walks the query blocks
+//    that attend block j (its own block and every block that kept it, from a
+//    reverse index), all query heads of the group, and accumulates
+//    dV^T = sum dO^T P and dK^T = sum Q^T dS in TMEM (M = head dim).
+// The cost is two recomputations of S and dP instead of one; in exchange
+// nothing is reduced through global memory and dq/dk/dv are deterministic.
+#include <cudaTypedefs.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace sas {
+
+bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 two warpgroups
+constexpr uint32_t kBox = 64 * 128;        // TMA box: 64 rows x 128 B
+constexpr uint32_t kTileAtom = 2 * kBox;   // 128 rows x 128 B (one 64-column half of a Q/dO tile)
+constexpr uint32_t kTile = 2 * kTileAtom;  // 128 rows x 256 B
+constexpr uint32_t kBlkAtom = kBox;        // 64 keys x 128 B
+constexpr uint32_t kBlk = 2 * kBlkAtom;    // 64 keys x 256 B
+
+// ------------------------------------------------------------------ shared
+struct Params {
+    int B, S, Hq, Hkv, G, K, NQB, ntg, n_items, ntile;
+    const int32_t* idx;
+    const int32_t* cnt;
+    const float* log_gate;
+    const float* lse;       // [B, Hq, S]
+    const float* Dr;        // [B, Hq, S]
+    const int32_t* rlist;   // [B, Hkv, NQB, NQB]: (i << 16) | slot, slot 0xFFFF = own block
+    const int32_t* rcount;  // [B, Hkv, NQB]
+    float scale2;           // sm_scale * log2(e)
+    float sm_scale;
+    __nv_bfloat16* dq;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* gsum;            // [B, Hkv, NQB, K]
+    int* status;
+};
+
+// ===================================================================== dq
+namespace dqk {
+
+constexpr uint32_t kOffQ = 0;                      // 2 tiles
+constexpr uint32_t kOffO = 2 * kTile;              // dO, 2 tiles
+constexpr uint32_t kOffKV = 4 * kTile;             // 2 stages x (K block, V block)
+constexpr int kNS = 2;
+constexpr uint32_t kStage = 2 * kBlk;
+constexpr uint32_t kOffBar = kOffKV + kNS * kStage;   // 192 KB
+constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
+
+struct Bars {
+    uint64_t qd_full, qd_empty;
+    uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
+    uint64_t s_full[2], ds_full[2], dq_full[2], dq_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct Item {
+    int b, h, i, tg, nt, c, nb;
+    long long row;
+};
+
+__device__ __forceinline__ Item item_of(const Params& p, int id) {
+    Item it;
+    const int per_i = p.B * p.Hkv * p.ntg;
+    it.i = p.NQB - 1 - id / per_i;
+    int r = id % per_i;
+    it.tg = r % p.ntg;
+    r /= p.ntg;
+    it.h = r % p.Hkv;
+    it.b = r / p.Hkv;
+    it.nt = (4 * it.tg + 2 < p.G) ? 2 : 1;
+    it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
+    it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));
+    it.nb = it.c + 1;
+    return it;
+}
+
+struct Blk {
+    int j;
+    bool valid, cur;
+    float bias2;
+};
+__device__ __forceinline__ Blk block_at(const Params& p, const Item& it, int k) {
+    Blk r;
+    if (k < it.c) {
+        const int j = __ldg(p.idx + it.row * p.K + k);
+        r.valid = (j >= 0 && j < it.i);
+        r.j = r.valid ? j : it.i;
+        r.cur = false;
+        r.bias2 = r.valid ? __ldg(p.log_gate + it.row * p.K + k) * kLog2e : 0.f;
+    } else {
+        r.j = it.i;
+        r.valid = true;
+        r.cur = true;
+        r.bias2 = 0.f;
+    }
+    return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
+          const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort = &bars->abort;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->qd_full, 1);
+        mbar_init(&bars->qd_empty, 1);
+        for (int s = 0; s < kNS; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->kv_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->ds_full[t], 128);
+            mbar_init(&bars->dq_full[t], 1);
+            mbar_init(&bars->dq_empty[t], 128);
+        }
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t sQ = smem_u32(smem + kOffQ), sO = smem_u32(smem + kOffO), sKV = smem_u32(smem + kOffKV);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t kv_it = 0, q_it = 0;
+            int last_it[kNS] = {-1, -1};
+            bool q_issued = false;
+            for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x) {
+                const Item it = item_of(p, id);
+                if (!mbar_wait(&bars->qd_empty, (q_it & 1) ^ 1, abort, p.status)) break;
+                mbar_expect_tx(&bars->qd_full, (uint32_t)it.nt * 8 * kBox);
+                for (int t = 0; t < it.nt; ++t)
+                    for (int s = 0; s < 2; ++s) {
+                        const int slot = 4 * it.tg + 2 * t + s;
+                        const int hq = it.h * p.G + (slot < p.G ? slot : 0);
+                        for (int a = 0; a < 2; ++a) {
+                            const uint32_t off = t * kTile + a * kTileAtom + s * kBox;
+                            tma_load_3d(smem + kOffQ + off, &map_q, &bars->qd_full, a * 64, hq, it.b * p.S + it.i * 64);
+                            tma_load_3d(smem + kOffO + off, &map_do, &bars->qd_full, a * 64, hq, it.b * p.S + it.i * 64);
+                        }
+                    }
+                q_issued = true;
+                ++q_it;
+                for (int k = 0; k < it.nb; ++k, ++kv_it) {
+                    const int st = kv_it % kNS;
+                    if (!mbar_wait(&bars->kv_empty[st], ((kv_it / kNS) & 1) ^ 1, abort, p.status)) break;
+                    const Blk bk = block_at(p, it, k);
+                    if (!bk.valid) flag_status(p.status, kStatusBadData);
+                    mbar_expect_tx(&bars->k_full[st], 2 * kBox);
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_3d(smem + kOffKV + st * kStage + a * kBlkAtom, &map_k, &bars->k_full[st], a * 64, it.h,
+                                    it.b * p.S + bk.j * 64);
+                    mbar_expect_tx(&bars->v_full[st], 2 * kBox);
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_3d(smem + kOffKV + st * kStage + kBlk + a * kBlkAtom, &map_v, &bars->v_full[st],
+                                    a * 64, it.h, it.b * p.S + bk.j * 64);
+                    last_it[st] = (int)kv_it;
+                }
+            }
+            if (*abort) {
+                volatile int no_abort = 0;
+                for (int s = 0; s < kNS; ++s)
+                    if (last_it[s] >= 0) {
+                        const uint32_t par = ((uint32_t)last_it[s] / kNS) & 1;
+                        mbar_wait(&bars->k_full[s], par, &no_abort, nullptr);
+                        mbar_wait(&bars->v_full[s], par, &no_abort, nullptr);
+                    }
+                if (q_issued) mbar_wait(&bars->qd_full, (q_it - 1) & 1, &no_abort, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(128, 64, false, false);
+            const uint32_t id_dq = idesc_bf16(128, kD, false, true);
+            uint32_t kv_it = 0, q_it = 0, ds_it[2] = {0, 0}, de_it[2] = {0, 0};
+            auto issue_sdp = [&](int t, int st) {
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t ao = t * kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                    const uint32_t bo = st * kStage + (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                    mma_ss(tmem + 256 * t, sw128_desc(sQ + ao, 16, 1024), sw128_desc(sKV + bo, 16, 1024), id_s, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t ao = t * kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                    const uint32_t bo = st * kStage + kBlk + (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                    mma_ss(tmem + 256 * t + 64, sw128_desc(sO + ao, 16, 1024), sw128_desc(sKV + bo, 16, 1024), id_s,
+                           kk > 0);
+                }
+            };
+            bool ok = true;
+            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
+                const Item it = item_of(p, id);
+                if (!(ok = mbar_wait(&bars->qd_full, q_it & 1, abort, p.status))) break;
+                ++q_it;
+                {
+                    const int st0 = kv_it % kNS;
+                    const uint32_t ph = (kv_it / kNS) & 1;
+                    if (!(ok = mbar_wait(&bars->k_full[st0], ph, abort, p.status))) break;
+                    if (!(ok = mbar_wait(&bars->v_full[st0], ph, abort, p.status))) break;
+                    tc_fence_after();
+                    for (int t = 0; t < it.nt; ++t) {
+                        issue_sdp(t, st0);
+                        mma_commit(&bars->s_full[t]);
+                    }
+                    if (it.nb == 1) mma_commit(&bars->qd_empty);
+                }
+                for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
+                    const int st = kv_it % kNS;
+                    const bool more = k + 1 < it.nb;
+                    const int st1 = (kv_it + 1) % kNS;
+                    const uint32_t ph1 = ((kv_it + 1) / kNS) & 1;
+                    for (int t = 0; t < it.nt && ok; ++t) {
+                        if (!(ok = mbar_wait(&bars->ds_full[t], ds_it[t] & 1, abort, p.status))) break;
+                        ++ds_it[t];
+                        if (k == 0) {
+                            if (!(ok = mbar_wait(&bars->dq_empty[t], (de_it[t] & 1) ^ 1, abort, p.status))) break;
+                            ++de_it[t];
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(tmem + 256 * t + 128, tmem + 256 * t + kk * 8,
+                                   sw128_desc(sKV + st * kStage + kk * 2048, kBlkAtom, 1024), id_dq,
+                                   (k > 0 || kk > 0) ? 1u : 0u);
+                        if (more) {
+                            if (t == 0) {
+                                if (!(ok = mbar_wait(&bars->k_full[st1], ph1, abort, p.status))) break;
+                                if (!(ok = mbar_wait(&bars->v_full[st1], ph1, abort, p.status))) break;
+                                tc_fence_after();
+                            }
+                            issue_sdp(t, st1);
+                            mma_commit(&bars->s_full[t]);
+                        } else {
+                            mma_commit(&bars->dq_full[t]);
+                        }
+                    }
+                    if (!ok) break;
+                    if (k + 2 == it.nb) mma_commit(&bars->qd_empty);
+                    mma_commit(&bars->kv_empty[st]);
+                }
+            }
+            mma_commit(&bars->drain);
+            volatile int no_abort = 0;
+            mbar_wait(&bars->drain, 0, &no_abort, nullptr);
+        }
+    } else {
+        const int t = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int slot_in_tile = row >> 6, r_in = row & 63;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_base + 256 * t;
+        const uint32_t tP = tS + 64;
+        const uint32_t tQ = tS + 128;
+        uint32_t s_it = 0, q_it = 0;
+        for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
+            const Item it = item_of(p, id);
+            if (t >= it.nt) continue;
+            const int slot = 4 * it.tg + 2 * t + slot_in_tile;
+            const bool row_ok = slot < p.G;
+            const int hq = it.h * p.G + (row_ok ? slot : 0);
+            const long long lrow = ((long long)it.b * p.Hq + hq) * p.S + (long long)it.i * 64 + r_in;
+            const float lse2 = p.lse[lrow] * kLog2e;
+            const float drow = p.Dr[lrow];
+            bool ok = true;
+            for (int k = 0; k < it.nb; ++k) {
+                const Blk bk = block_at(p, it, k);
+                if (!(ok = mbar_wait(&bars->s_full[t], s_it & 1, abort, p.status))) break;
+                ++s_it;
+                tc_fence_after();
+                uint32_t sv[2][32], pv[2][32];
+                tmem_ld32(tS, sv[0]);
+                tmem_ld32(tS + 32, sv[1]);
+                tmem_ld32(tP, pv[0]);
+                tmem_ld32(tP + 32, pv[1]);
+                tmem_wait_ld();
+                const float off = bk.bias2 - lse2;
+                float gs = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float d2[2];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int u = 2 * e + q;
+                        const bool live = row_ok && bk.valid && !(bk.cur && u > r_in);
+                        const float s = __uint_as_float(sv[u >> 5][u & 31]);
+                        const float dp = __uint_as_float(pv[u >> 5][u & 31]);
+                        const float pr = live ? exp2f(fmaf(s, p.scale2, off)) : 0.f;
+                        const float ds = pr * (dp - drow);
+                        gs += ds;
+                        d2[q] = ds * p.sm_scale;
+                    }
+                    pk[e] = pack_bf16x2(d2[0], d2[1]);
+                }
+                tmem_st32(tS, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->ds_full[t]);
+                if (!bk.cur && bk.valid) {
+                    gs = warp_sum(gs);
+                    if (lane == 0) atomicAdd(p.gsum + it.row * p.K + k, gs);
+                }
+            }
+            if (!ok) break;
+            if (!mbar_wait(&bars->dq_full[t], q_it & 1, abort, p.status)) break;
+            ++q_it;
+            tc_fence_after();
+            const long long orow = ((long long)it.b * p.S + (long long)it.i * 64 + r_in) * p.Hq + hq;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t ov[32];
+                tmem_ld32(tQ + q4 * 32, ov);
+                tmem_wait_ld();
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.dq + orow * kD + q4 * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]), __uint_as_float(ov[8 * v4 + 1]));
+                        w.y = pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]), __uint_as_float(ov[8 * v4 + 3]));
+                        w.z = pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]), __uint_as_float(ov[8 * v4 + 5]));
+                        w.w = pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]), __uint_as_float(ov[8 * v4 + 7]));
+                        dst[v4] = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->dq_empty[t]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace dqk
+
+// ==================================================================== dk, dv
+namespace dkv {
+
+constexpr uint32_t kOffK = 0;                      // K_j: 64 keys x 256 B
+constexpr uint32_t kOffV = kBlk;                   // V_j
+constexpr uint32_t kOffStage = 2 * kBlk;           // 2 stages x (Q tile, dO tile)
+constexpr int kNS = 2;
+constexpr uint32_t kStage = 2 * kTile;
+constexpr uint32_t kOffPS = kOffStage + kNS * kStage;    // per warpgroup: P (128 x 64 bf16), dS
+constexpr uint32_t kPSBuf = 128 * 128;                    // 16 KB
+constexpr uint32_t kOffBar = kOffPS + 2 * 2 * kPSBuf;     // 224 KB
+constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
+
+struct Bars {
+    uint64_t kv_full, kv_empty;
+    uint64_t qd_full[kNS], qd_empty[kNS];
+    uint64_t s_full[2], pds_full[2], pds_empty[2];
+    uint64_t acc_full, acc_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void item_of(const Params& p, int id, int& b, int& h, int& j, long long& bh) {
+    j = id % p.NQB;
+    const int r = id / p.NQB;
+    h = r % p.Hkv;
+    b = r / p.Hkv;
+    bh = (long long)b * p.Hkv + h;
+}
+
+__device__ __forceinline__ int n_entries(const Params& p, long long bh, int j) {
+    const int n = p.rcount[bh * p.NQB + j];
+    return max(1, min(n, p.NQB - j));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
+           const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort = &bars->abort;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        mbar_init(&bars->kv_empty, 1);
+        for (int s = 0; s < kNS; ++s) {
+            mbar_init(&bars->qd_full[s], 1);
+            mbar_init(&bars->qd_empty[s], 1);
+        }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&bars->s_full[w], 1);
+            mbar_init(&bars->pds_full[w], 128);
+            mbar_init(&bars->pds_empty[w], 1);
+        }
+        mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->acc_empty, 256);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t s_base = smem_u32(smem);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t item_it = 0, qd_it = 0;
+            int last_it[kNS] = {-1, -1};
+            bool kv_issued = false;
+            for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x, ++item_it) {
+                int b, h, j;
+                long long bh;
+                item_of(p, id, b, h, j, bh);
+                const int n = n_entries(p, bh, j);
+                if (!mbar_wait(&bars->kv_empty, (item_it & 1) ^ 1, abort, p.status)) break;
+                mbar_expect_tx(&bars->kv_full, 4 * kBox);
+                for (int a = 0; a < 2; ++a) {
+                    tma_load_3d(smem + kOffK + a * kBlkAtom, &map_k, &bars->kv_full, a * 64, h, b * p.S + j * 64);
+                    tma_load_3d(smem + kOffV + a * kBlkAtom, &map_v, &bars->kv_full, a * 64, h, b * p.S + j * 64);
+                }
+                kv_issued = true;
+                const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
+                for (int e = 0; e < n && !*abort; ++e) {
+                    int i = __ldg(list + e) >> 16;
+                    if (i < j || i >= p.NQB) {
+                        flag_status(p.status, kStatusBadData);
+                        i = j;
+                    }
+                    for (int t = 0; t < p.ntile; ++t, ++qd_it) {
+                        const int st = qd_it % kNS;
+                        if (!mbar_wait(&bars->qd_empty[st], ((qd_it / kNS) & 1) ^ 1, abort, p.status)) break;
+                        mbar_expect_tx(&bars->qd_full[st], 8 * kBox);
+                        for (int s = 0; s < 2; ++s) {
+                            const int slot = 2 * t + s;
+                            const int hq = h * p.G + (slot < p.G ? slot : 0);
+                            for (int a = 0; a < 2; ++a) {
+                                const uint32_t off = kOffStage + st * kStage + a * kTileAtom + s * kBox;
+                                tma_load_3d(smem + off, &map_q, &bars->qd_full[st], a * 64, hq, b * p.S + i * 64);
+                                tma_load_3d(smem + off + kTile, &map_do, &bars->qd_full[st], a * 64, hq,
+                                            b * p.S + i * 64);
+                            }
+                        }
+                        last_it[st] = (int)qd_it;
+                    }
+                }
+            }
+            if (*abort) {
+                volatile int no_abort = 0;
+                for (int s = 0; s < kNS; ++s)
+                    if (last_it[s] >= 0)
+                        mbar_wait(&bars->qd_full[s], ((uint32_t)last_it[s] / kNS) & 1, &no_abort, nullptr);
+                if (kv_issued) mbar_wait(&bars->kv_full, (item_it - 1) & 1, &no_abort, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(128, 64, false, false);
+            const uint32_t id_t = idesc_bf16(128, 64, true, true);
+            uint32_t item_it = 0, qd_it = 0, pds_it[2] = {0, 0};
+            bool ok = true;
+            // dV^T += dO^T P, dK^T += Q^T dS for step m (stage st, warpgroup w)
+            auto dvdk = [&](int m, int st, uint32_t item_parity) -> bool {
+                const int w = m & 1;
+                if (!mbar_wait(&bars->pds_full[w], pds_it[w] & 1, abort, p.status)) return false;
+                ++pds_it[w];
+                if (m == 0 && !mbar_wait(&bars->acc_empty, item_parity ^ 1, abort, p.status)) return false;
+                tc_fence_after();
+                const uint32_t sq = s_base + kOffStage + st * kStage;
+                const uint32_t sp = s_base + kOffPS + w * 2 * kPSBuf;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + 256, sw128_desc(sq + kTile + kk * 2048, kTileAtom, 1024),
+                           sw128_desc(sp + kk * 2048, kPSBuf, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + 320, sw128_desc(sq + kk * 2048, kTileAtom, 1024),
+                           sw128_desc(sp + kPSBuf + kk * 2048, kPSBuf, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars->qd_empty[st]);
+                mma_commit(&bars->pds_empty[w]);
+                return true;
+            };
+            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+                int b, h, j;
+                long long bh;
+                item_of(p, id, b, h, j, bh);
+                const int N = n_entries(p, bh, j) * p.ntile;
+                if (!(ok = mbar_wait(&bars->kv_full, item_it & 1, abort, p.status))) break;
+                tc_fence_after();
+                int prev_st = 0;
+                for (int m = 0; m < N && ok; ++m, ++qd_it) {
+                    const int st = qd_it % kNS;
+                    const int w = m & 1;
+                    if (!(ok = mbar_wait(&bars->qd_full[st], (qd_it / kNS) & 1, abort, p.status))) break;
+                    tc_fence_after();
+                    const uint32_t sq = s_base + kOffStage + st * kStage;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                        const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                        mma_ss(tmem + 128 * w, sw128_desc(sq + ao, 16, 1024), sw128_desc(s_base + kOffK + bo, 16, 1024),
+                               id_s, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ao = kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                        const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                        mma_ss(tmem + 128 * w + 64, sw128_desc(sq + ao, 16, 1024),
+                               sw128_desc(s_base + kOffV + bo, 16, 1024), id_s, kk > 0);
+                    }
+                    mma_commit(&bars->s_full[w]);
+                    if (m > 0 && !(ok = dvdk(m - 1, prev_st, item_it & 1))) break;
+                    prev_st = st;
+                }
+                if (!ok) break;
+                if (!(ok = dvdk(N - 1, prev_st, item_it & 1))) break;
+                mma_commit(&bars->kv_empty);
+                mma_commit(&bars->acc_full);
+            }
+            mma_commit(&bars->drain);
+            volatile int no_abort = 0;
+            mbar_wait(&bars->drain, 0, &no_abort, nullptr);
+        }
+    } else {
+        const int w = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int r_in = row & 63;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_base + 128 * w;
+        uint8_t* bufP = smem + kOffPS + w * 2 * kPSBuf;
+        uint8_t* bufS = bufP + kPSBuf;
+        uint32_t s_it = 0, pe_it = 0, item_it = 0;
+        bool ok = true;
+        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+            int b, h, j;
+            long long bh;
+            item_of(p, id, b, h, j, bh);
+            const int N = n_entries(p, bh, j) * p.ntile;
+            const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
+            for (int m = w; m < N; m += 2) {
+                const int e = m / p.ntile, t = m % p.ntile;
+                const int ent = __ldg(list + e);
+                int i = ent >> 16;
+                const int slot = ent & 0xFFFF;
+                bool valid = i >= j && i < p.NQB;
+                if (!valid) i = j;
+                const bool cur = (i == j);
+                float bias2 = 0.f;
+                if (!cur) {
+                    const long long srow = bh * p.NQB + i;
+                    valid = valid && slot < p.K && __ldg(p.idx + srow * p.K + slot) == j;
+                    bias2 = valid ? __ldg(p.log_gate + srow * p.K + slot) * kLog2e : 0.f;
+                }
+                const int hs = 2 * t + (row >> 6);
+                const bool row_ok = valid && hs < p.G;
+                const int hq = h * p.G + (hs < p.G ? hs : 0);
+                const long long lrow = ((long long)b * p.Hq + hq) * p.S + (long long)i * 64 + r_in;
+                const float lse2 = p.lse[lrow] * kLog2e;
+                const float drow = p.Dr[lrow];
+                if (!(ok = mbar_wait(&bars->s_full[w], s_it & 1, abort, p.status))) break;
+                ++s_it;
+                tc_fence_after();
+                // the MMA of this warpgroup's previous step has finished reading the buffers
+                if (!(ok = mbar_wait(&bars->pds_empty[w], (pe_it & 1) ^ 1, abort, p.status))) break;
+                ++pe_it;
+                const float off = bias2 - lse2;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {           // keys [32 hf, 32 hf + 32)
+                    uint32_t sv[32], pv[32];
+                    tmem_ld32(tS + 32 * hf, sv);
+                    tmem_ld32(tS + 64 + 32 * hf, pv);
+                    tmem_wait_ld();
+                    uint32_t pp[16], dd[16];
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        float pr2[2], ds2[2];
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int u = 32 * hf + 2 * e2 + q;
+                            const bool live = row_ok && !(cur && u > r_in);
+                            pr2[q] = live ? exp2f(fmaf(__uint_as_float(sv[2 * e2 + q]), p.scale2, off)) : 0.f;
+                            ds2[q] = pr2[q] * (__uint_as_float(pv[2 * e2 + q]) - drow) * p.sm_scale;
+                        }
+                        pp[e2] = pack_bf16x2(pr2[0], pr2[1]);
+                        dd[e2] = pack_bf16x2(ds2[0], ds2[1]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        *reinterpret_cast<uint4*>(bufP + sw128_offset(row, 4 * hf + c)) =
+                            make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+                        *reinterpret_cast<uint4*>(bufS + sw128_offset(row, 4 * hf + c)) =
+                            make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars->pds_full[w]);
+            }
+            if (!ok) break;
+            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim index)
+            if (!(ok = mbar_wait(&bars->acc_full, item_it & 1, abort, p.status))) break;
+            tc_fence_after();
+            {
+                const int d = row;
+                __nv_bfloat16* out = (w == 0 ? p.dv : p.dk) + ((long long)b * p.S + (long long)j * 64) * p.Hkv * kD +
+                                     (long long)h * kD + d;
+                const long long key_stride = (long long)p.Hkv * kD;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + 256 + 64 * w + 32 * hf, v);
+                    tmem_wait_ld();
+                    __nv_bfloat16* o2 = out + 32 * hf * key_stride;
+#pragma unroll 8
+                    for (int u = 0; u < 32; ++u) o2[u * key_stride] = __float2bfloat16_rn(__uint_as_float(v[u]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->acc_empty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace dkv
+
+// ================================================================ helpers
+__global__ void dot_rows_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                long long rows, int S, int Hq, float* __restrict__ Dr) {
+    // one warp per (b, t, hq) row of 128; Dr as [B, Hq, S]
+    const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= rows) return;
+    const uint2 a = reinterpret_cast<const uint2*>(o + w * kD)[lane];
+    const uint2 c = reinterpret_cast<const uint2*>(dout + w * kD)[lane];
+    float2 a0 = bf16x2_to_f32(a.x), a1 = bf16x2_to_f32(a.y), c0 = bf16x2_to_f32(c.x), c1 = bf16x2_to_f32(c.y);
+    float acc = a0.x * c0.x + a0.y * c0.y + a1.x * c1.x + a1.y * c1.y;
+    acc = warp_sum(acc);
+    if (lane == 0) {
+        const int hq = (int)(w % Hq);
+        const long long bt = w / Hq;
+        const long long b = bt / S, t = bt % S;
+        Dr[(b * Hq + hq) * S + t] = acc;
+    }
+}
+
+__global__ void rev_fill_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int rows, int NQB,
+                                int K, int16_t* __restrict__ slotmap) {
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int i = (int)(row % NQB);
+    const long long bh = row / NQB;
+    const int c = max(0, min(cnt[row], min(K, i)));
+    for (int k = lane; k < c; k += 32) {
+        const int j = idx[row * K + k];
+        if (j >= 0 && j < i) slotmap[(bh * NQB + j) * NQB + i] = (int16_t)(k + 1);
+    }
+}
+
+__global__ void rev_list_kernel(const int16_t* __restrict__ slotmap, int rows, int NQB, int32_t* __restrict__ rlist,
+                                int32_t* __restrict__ rcount) {
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // (bh, j)
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int j = (int)(row % NQB);
+    int32_t* list = rlist + row * NQB;
+    const int16_t* sm = slotmap + row * NQB;
+    if (lane == 0) list[0] = (j << 16) | 0xFFFF;
+    int n = 1;
+    for (int i0 = j + 1; i0 < NQB; i0 += 32) {
+        const int i = i0 + lane;
+        const int v = (i < NQB) ? sm[i] : 0;
+        const unsigned ball = __ballot_sync(0xffffffffu, v != 0);
+        if (v != 0) list[n + __popc(ball & ((1u << lane) - 1u))] = (i << 16) | (v - 1);
+        n += __popc(ball);
+    }
+    if (lane == 0) rcount[row] = n;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Ws {
+    float* Dr;
+    float* gsum;
+    int16_t* slotmap;
+    int32_t* rlist;
+    int32_t* rcount;
+};
+
+Ws carve(void* w, int B, int S, int Hq, int Hkv, int K) {
+    const int NQB = S / 64;
+    char* p = static_cast<char*>(w);
+    Ws r;
+    r.Dr = reinterpret_cast<float*>(p);
+    p += align256(sizeof(float) * (size_t)B * Hq * S);
+    r.gsum = reinterpret_cast<float*>(p);
+    p += align256(sizeof(float) * (size_t)B * Hkv * NQB * (size_t)(K > 0 ? K : 1));
+    r.slotmap = reinterpret_cast<int16_t*>(p);
+    p += align256(sizeof(int16_t) * (size_t)B * Hkv * NQB * NQB);
+    r.rlist = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * (size_t)B * Hkv * NQB * NQB);
+    r.rcount = reinterpret_cast<int32_t*>(p);
+    return r;
+}
+
+}  // namespace
+
+size_t bwd_sm100_workspace(int B, int S, int Hq, int Hkv, int K) {
+    const int NQB = S / 64;
+    return align256(sizeof(float) * (size_t)B * Hq * S) +
+           align256(sizeof(float) * (size_t)B * Hkv * NQB * (size_t)(K > 0 ? K : 1)) +
+           align256(sizeof(int16_t) * (size_t)B * Hkv * NQB * NQB) +
+           align256(sizeof(int32_t) * (size_t)B * Hkv * NQB * NQB) + align256(sizeof(int32_t) * (size_t)B * Hkv * NQB);
+}
+
+cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
+    const AttnArgs& a = bw.a;
+    const int NQB = a.S / 64, G = a.Hq / a.Hkv;
+    const long long rows = (long long)a.B * a.S;
+    CUtensorMap mq, mdo, mk, mv;
+    if (!make_head_map(&mq, a.q, rows, a.Hq, kD) || !make_head_map(&mdo, bw.dout, rows, a.Hq, kD) ||
+        !make_head_map(&mk, a.k, rows, a.Hkv, kD) || !make_head_map(&mv, a.v, rows, a.Hkv, kD))
+        return cudaErrorInvalidValue;
+    Ws ws = carve(bw.workspace, a.B, a.S, a.Hq, a.Hkv, a.K);
+    cudaError_t e;
+    const int bhq = a.B * a.Hkv * NQB;
+    if ((e = cudaMemsetAsync(ws.gsum, 0, sizeof(float) * (size_t)bhq * (a.K > 0 ? a.K : 1), st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(ws.slotmap, 0, sizeof(int16_t) * (size_t)bhq * NQB, st)) != cudaSuccess) return e;
+    const long long drows = rows * a.Hq;
+    dot_rows_kernel<<<(unsigned)((drows + 7) / 8), 256, 0, st>>>((const __nv_bfloat16*)bw.o,
+                                                                 (const __nv_bfloat16*)bw.dout, drows, a.S, a.Hq, ws.Dr);
+    rev_fill_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(a.idx, a.cnt, bhq, NQB, a.K, ws.slotmap);
+    rev_list_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(ws.slotmap, bhq, NQB, ws.rlist, ws.rcount);
+    count_launches(3);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    Params p;
+    p.B = a.B;
+    p.S = a.S;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.G = G;
+    p.K = a.K;
+    p.NQB = NQB;
+    p.ntg = ((G + 1) / 2 + 1) / 2;
+    p.ntile = (G + 1) / 2;
+    p.idx = a.idx;
+    p.cnt = a.cnt;
+    p.log_gate = a.log_gate;
+    p.lse = bw.lse;
+    p.Dr = ws.Dr;
+    p.rlist = ws.rlist;
+    p.rcount = ws.rcount;
+    p.scale2 = a.sm_scale * kLog2e;
+    p.sm_scale = a.sm_scale;
+    p.dq = static_cast<__nv_bfloat16*>(bw.dq);
+    p.dk = static_cast<__nv_bfloat16*>(bw.dk);
+    p.dv = static_cast<__nv_bfloat16*>(bw.dv);
+    p.gsum = ws.gsum;
+    p.status = a.status;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+    p.n_items = a.B * a.Hkv * NQB * p.ntg;
+    if ((e = cudaFuncSetAttribute(dqk::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dqk::kSmem)) !=
+        cudaSuccess)
+        return e;
+    dqk::dq_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, dqk::kSmem, st>>>(mq, mdo, mk, mv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    p.n_items = a.B * a.Hkv * NQB;
+    if ((e = cudaFuncSetAttribute(dkv::dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkv::kSmem)) !=
+        cudaSuccess)
+        return e;
+    dkv::dkv_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, dkv::kSmem, st>>>(mq, mdo, mk, mv, p);
+    count_launches(2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_ds_finalize(bw.s, bw.ld_s, bw.lse_s, a.idx, a.cnt, ws.gsum, a.B, a.Hkv, NQB, a.K, bw.ds, st);
+}
+
+}  // namespace sas

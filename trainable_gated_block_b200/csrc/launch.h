@@ -42,6 +42,13 @@ struct BwdArgs {
 };
 size_t bwd_simt_workspace(int B, int S, int Hq, int Hkv, int D, int K);
 cudaError_t launch_bwd_simt(const BwdArgs& b, bool bf16, cudaStream_t st);
+// bf16, D = 128: tcgen05 tensor-core path.
+size_t bwd_sm100_workspace(int B, int S, int Hq, int Hkv, int K);
+cudaError_t launch_bwd_sm100(const BwdArgs& b, cudaStream_t st);
+// ds from the per-block gate gradients gsum [B, Hkv, NQB, K].
+cudaError_t launch_ds_finalize(const float* s, int ld_s, const float* lse_s, const int32_t* idx,
+                               const int32_t* cnt, const float* gsum, int B, int Hkv, int NQB, int K,
+                               float* ds, cudaStream_t st);
 
 // Decode.
 struct DecodeArgs {

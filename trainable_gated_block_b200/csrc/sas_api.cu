@@ -135,6 +135,7 @@ size_t sas_attn_bwd_workspace_size(sas_dtype dtype, int B, int S, int Hq, int Hk
     if ((dtype != SAS_F32 && dtype != SAS_BF16) || B <= 0 || S <= 0 || S % 64 || Hq <= 0 || Hkv <= 0 ||
         Hq % Hkv || (D != 64 && D != 128) || K < 0)
         return 0;
+    if (dtype == SAS_BF16 && D == 128) return sas::bwd_sm100_workspace(B, S, Hq, Hkv, K);
     return sas::bwd_simt_workspace(B, S, Hq, Hkv, D, K);
 }
 
@@ -159,7 +160,9 @@ sas_status sas_attn_bwd(sas_dtype dtype, const void* q, const void* k, const voi
     if (!st) return fail(SAS_ERR_CUDA, "sas_attn_bwd: no CUDA device");
     sas::BwdArgs b{{q, k, v, B, S, Hq, Hkv, D, K, idx, cnt, log_gate, sm_scale, st},
                    o, dout, lse, s, ld_s, lse_s, dq, dk, dv, ds, workspace, ws_bytes};
-    cudaError_t e = sas::launch_bwd_simt(b, dtype == SAS_BF16, static_cast<cudaStream_t>(stream));
+    cudaError_t e = (dtype == SAS_BF16 && D == 128)
+                        ? sas::launch_bwd_sm100(b, static_cast<cudaStream_t>(stream))
+                        : sas::launch_bwd_simt(b, dtype == SAS_BF16, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "sas_attn_bwd");
 }
 

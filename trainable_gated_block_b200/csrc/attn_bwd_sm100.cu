@@ -26,9 +26,6 @@
 #include "sm100.cuh"
 
 namespace sas {
-
-bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D);
-
 namespace {
 
 using namespace sm100;

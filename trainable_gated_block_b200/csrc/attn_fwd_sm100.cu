@@ -7,24 +7,23 @@
 //
 // Work item = (batch b, KV head h, query block i, head group tg): up to two
 // 128-row Q tiles, each tile = 2 query heads x the 64 rows of block i. All
-// query heads of a GQA group share the same kept blocks, so one K/V tile
-// feeds both Q tiles. Persistent grid; items in order of decreasing cost.
+// query heads of a GQA group share the kept blocks, so one K/V block feeds
+// both Q tiles. Persistent grid; items in order of decreasing cost.
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: Q tiles once per item, then K/V of two kept
-//               blocks (128 keys) per step into a 2-stage ring, 128B-swizzled.
-//   warp 1      TMEM owner and tcgen05 MMA issuer (one thread):
-//               S_t = Q_t K^T into TMEM, then O_t += P_t V with P read from TMEM.
-//   warps 2-5   softmax for Q tile 0, warps 6-9 for Q tile 1: each thread
-//               owns one row (one TMEM lane); adds the block's log-gate to
-//               the logits, masks the diagonal block causally, keeps an
-//               online max/sum in the log2 domain, writes P (bf16) over S in
-//               TMEM, rescales O in TMEM only when the max grows by > 2^8,
-//               and finally writes o and the row LSE.
-// TMEM (512 columns): S/P of tile t at [128t, 128t+128), O of tile t at
-// [256+128t, 256+128t+128).
-#include <cudaTypedefs.h>
-
+// One step = one kept block (64 keys). Warp roles (320 threads):
+//   warp 0      TMA producer: the Q tiles once per item, then K and V of one
+//               block per step into a 4-stage ring (128B-swizzled).
+//   warp 1      TMEM owner and tcgen05 issuer (one thread): S_t = Q_t K^T
+//               into one of two S buffers per tile, O_t += P_t V with P read
+//               from TMEM. S of step j+2 is issued as soon as PV of step j is,
+//               so the softmax of step j+1 never waits for an MMA.
+//   warps 2-5   softmax of Q tile 0, warps 6-9 of tile 1: one row per thread
+//               (one TMEM lane); logits = sm_scale q.k + log-gate in the log2
+//               domain, causal mask on the diagonal block, running max/sum;
+//               P (bf16) over the consumed S buffer; O in TMEM rescaled only
+//               when the max grows by more than 2^8; final o and row LSE.
+// TMEM (512 columns): tile t owns [256t, 256t+256): S buffers at +0 and +64
+// (64 columns each, P overwrites the first 32), O at +128.
 #include "launch.h"
 #include "sm100.cuh"
 
@@ -34,24 +33,32 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kNS = 2;                              // K/V stages
+constexpr int kNS = 4;                              // K/V stages (one block each)
 constexpr int kThreads = 320;
 constexpr uint32_t kBox = 64 * 128;                 // one TMA box: 64 rows x 128 B
 constexpr uint32_t kQAtom = 2 * kBox;               // 128 rows x 128 B
 constexpr uint32_t kQTile = 2 * kQAtom;             // 128 rows x 256 B
-constexpr uint32_t kKVAtom = 2 * kBox;              // 128 keys x 128 B
-constexpr uint32_t kKVTile = 2 * kKVAtom;
+constexpr uint32_t kBlkAtom = kBox;                 // 64 keys x 128 B
+constexpr uint32_t kBlk = 2 * kBlkAtom;             // 64 keys x 256 B
+constexpr uint32_t kStage = 2 * kBlk;               // K block + V block
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = 2 * kQTile;                          // 64 KB
-constexpr uint32_t kOffV = kOffK + kNS * kKVTile;
-constexpr uint32_t kOffBar = kOffV + kNS * kKVTile;             // 192 KB
-constexpr uint32_t kSmemBytes = kOffBar + 1024 + 1024;          // + barriers + alignment slack
-constexpr float kRescaleThreshold = 8.0f;           // log2 units: rescale O when the max grows by > 256x
+constexpr uint32_t kOffKV = 2 * kQTile;                         // 64 KB
+constexpr uint32_t kOffBar = kOffKV + kNS * kStage;             // 192 KB
+constexpr uint32_t kSmemBytes = kOffBar + 1024 + 1024;
+constexpr float kRescaleThreshold = 8.0f;           // log2 units
+
+struct Meta {            // one block of an item's list
+    int j;               // block index actually loaded
+    float bias2;         // log-gate * log2(e) (0 on the current block)
+    int live;            // 0: masked out entirely (bad index)
+    int cur;             // 1: the query's own block (causal mask)
+};
 
 struct Bars {
     uint64_t q_full, q_empty;
     uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
-    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+    uint64_t s_full[2][2], p_full[2][2];
+    uint64_t o_done[2], o_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -69,9 +76,8 @@ struct Params {
 };
 
 struct Item {
-    int b, h, i, tg, nt, c, nb, ns;
-    const int32_t* sel;
-    const float* gate;
+    int b, h, i, tg, nt, c, nb;
+    long long row;
 };
 
 __device__ __forceinline__ Item item_of(const Params& p, int id) {
@@ -84,40 +90,30 @@ __device__ __forceinline__ Item item_of(const Params& p, int id) {
     it.h = r % p.Hkv;
     it.b = r / p.Hkv;
     it.nt = (4 * it.tg + 2 < p.G) ? 2 : 1;
-    const long long row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
-    int c = p.cnt[row];
-    const int cmax = min(p.K, it.i);
-    c = max(0, min(c, cmax));
-    it.c = c;
-    it.nb = c + 1;
-    it.ns = (it.nb + 1) >> 1;
-    it.sel = p.idx + row * p.K;
-    it.gate = p.log_gate + row * p.K;
+    it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
+    it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));
+    it.nb = it.c + 1;
     return it;
 }
 
-// Block k of the item's list (kept blocks ascending, then the current block).
+// Block k of the item's list: kept blocks ascending, then the current block.
 // An out-of-range index is replaced by the current block, fully masked.
-struct Blk {
-    int j;
-    bool valid, cur;
-    float bias2;        // log-gate in log2 units
-};
-__device__ __forceinline__ Blk block_at(const Item& it, int k) {
-    Blk r;
+__device__ __forceinline__ Meta meta_at(const Params& p, const Item& it, int k) {
+    Meta m;
     if (k < it.c) {
-        const int j = __ldg(it.sel + k);
-        r.valid = (j >= 0 && j < it.i);
-        r.j = r.valid ? j : it.i;
-        r.cur = false;
-        r.bias2 = r.valid ? __ldg(it.gate + k) * kLog2e : 0.f;
+        const int j = __ldg(p.idx + it.row * p.K + k);
+        const bool ok = j >= 0 && j < it.i;
+        m.j = ok ? j : it.i;
+        m.bias2 = ok ? __ldg(p.log_gate + it.row * p.K + k) * kLog2e : 0.f;
+        m.live = ok;
+        m.cur = 0;
     } else {
-        r.j = it.i;
-        r.valid = true;
-        r.cur = true;
-        r.bias2 = 0.f;
+        m.j = it.i;
+        m.bias2 = 0.f;
+        m.live = 1;
+        m.cur = 1;
     }
-    return r;
+    return m;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -138,9 +134,11 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(&bars->s_full[t], 1);
-            mbar_init(&bars->p_full[t], 128);
-            mbar_init(&bars->o_full[t], 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&bars->s_full[t][b], 1);
+                mbar_init(&bars->p_full[t][b], 128);
+            }
+            mbar_init(&bars->o_done[t], 1);
             mbar_init(&bars->o_empty[t], 128);
         }
         mbar_init(&bars->drain, 1);
@@ -161,18 +159,17 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const uint32_t sQ = smem_u32(smem + kOffQ);
-    const uint32_t sK = smem_u32(smem + kOffK);
-    const uint32_t sV = smem_u32(smem + kOffV);
+    const uint32_t sKV = smem_u32(smem + kOffKV);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t kv_it = 0, q_it = 0;
-            int last_stage_it[kNS] = {-1, -1};
+            int last_it[kNS] = {-1, -1, -1, -1};
             bool q_issued = false;
             for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x) {
                 const Item it = item_of(p, id);
-                if (p.cnt[((long long)it.b * p.Hkv + it.h) * p.NQB + it.i] != it.c) flag_status(p.status, kStatusBadData);
+                if (p.cnt[it.row] != it.c) flag_status(p.status, kStatusBadData);
                 if (!mbar_wait(&bars->q_empty, (q_it & 1) ^ 1, abort, p.status)) break;
                 mbar_expect_tx(&bars->q_full, (uint32_t)it.nt * 4 * kBox);
                 for (int t = 0; t < it.nt; ++t)
@@ -185,61 +182,45 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 q_issued = true;
                 ++q_it;
-                for (int j = 0; j < it.ns; ++j, ++kv_it) {
+                for (int k = 0; k < it.nb; ++k, ++kv_it) {
                     const int st = kv_it % kNS;
                     if (!mbar_wait(&bars->kv_empty[st], ((kv_it / kNS) & 1) ^ 1, abort, p.status)) break;
-                    const int nblk = (2 * j + 1 < it.nb) ? 2 : 1;
-                    mbar_expect_tx(&bars->k_full[st], (uint32_t)nblk * 2 * kBox);
-                    for (int bl = 0; bl < nblk; ++bl) {
-                        const Blk bk = block_at(it, 2 * j + bl);
-                        if (!bk.valid) flag_status(p.status, kStatusBadData);
-                        for (int a = 0; a < 2; ++a)
-                            tma_load_3d(smem + kOffK + st * kKVTile + a * kKVAtom + bl * kBox, &map_k,
-                                        &bars->k_full[st], a * 64, it.h, it.b * p.S + bk.j * 64);
-                    }
-                    mbar_expect_tx(&bars->v_full[st], (uint32_t)nblk * 2 * kBox);
-                    for (int bl = 0; bl < nblk; ++bl) {
-                        const Blk bk = block_at(it, 2 * j + bl);
-                        for (int a = 0; a < 2; ++a)
-                            tma_load_3d(smem + kOffV + st * kKVTile + a * kKVAtom + bl * kBox, &map_v,
-                                        &bars->v_full[st], a * 64, it.h, it.b * p.S + bk.j * 64);
-                    }
-                    last_stage_it[st] = (int)kv_it;
+                    const Meta m = meta_at(p, it, k);
+                    if (!m.live) flag_status(p.status, kStatusBadData);
+                    mbar_expect_tx(&bars->k_full[st], 2 * kBox);
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_3d(smem + kOffKV + st * kStage + a * kBlkAtom, &map_k, &bars->k_full[st], a * 64,
+                                    it.h, it.b * p.S + m.j * 64);
+                    mbar_expect_tx(&bars->v_full[st], 2 * kBox);
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_3d(smem + kOffKV + st * kStage + kBlk + a * kBlkAtom, &map_v, &bars->v_full[st],
+                                    a * 64, it.h, it.b * p.S + m.j * 64);
+                    last_it[st] = (int)kv_it;
                 }
             }
             if (*abort) {
-                // let every copy this thread started land before the CTA exits
+                volatile int no_abort = 0;
                 for (int s = 0; s < kNS; ++s)
-                    if (last_stage_it[s] >= 0) {
-                        const uint32_t par = ((uint32_t)last_stage_it[s] / kNS) & 1;
-                        volatile int no_abort = 0;
+                    if (last_it[s] >= 0) {
+                        const uint32_t par = ((uint32_t)last_it[s] / kNS) & 1;
                         mbar_wait(&bars->k_full[s], par, &no_abort, nullptr);
                         mbar_wait(&bars->v_full[s], par, &no_abort, nullptr);
                     }
-                if (q_issued) {
-                    volatile int no_abort = 0;
-                    mbar_wait(&bars->q_full, (q_it - 1) & 1, &no_abort, nullptr);
-                }
+                if (q_issued) mbar_wait(&bars->q_full, (q_it - 1) & 1, &no_abort, nullptr);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_pv = idesc_bf16(128, kD, false, true);
-            uint32_t kv_it = 0, q_it = 0, p_it[2] = {0, 0}, oe_it[2] = {0, 0};
-            auto issue_s = [&](int t, int st, int nk) {
-                const uint32_t idesc = idesc_bf16(128, nk, false, false);
+            const uint32_t id_s = idesc_bf16(128, 64, false, false);
+            const uint32_t id_pv = idesc_bf16(128, kD, false, true);
+            uint32_t kv_it = 0, q_it = 0, p_it[2][2] = {{0, 0}, {0, 0}}, oe_it[2] = {0, 0};
+            auto issue_s = [&](int t, int st, int buf) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint64_t a = sw128_desc(sQ + t * kQTile + (kk >> 2) * kQAtom + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = sw128_desc(sK + st * kKVTile + (kk >> 2) * kKVAtom + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tmem + t * 128, a, b, idesc, kk > 0);
-                }
-            };
-            auto issue_pv = [&](int t, int st, int nk, bool acc) {
-                for (int kk = 0; kk < nk / 16; ++kk) {
-                    const uint64_t b = sw128_desc(sV + st * kKVTile + kk * 2048, kKVAtom, 1024);
-                    mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    const uint64_t b = sw128_desc(sKV + st * kStage + (kk >> 2) * kBlkAtom + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tmem + 256 * t + 64 * buf, a, b, id_s, kk > 0);
                 }
             };
             bool ok = true;
@@ -248,52 +229,54 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 if (!(ok = mbar_wait(&bars->q_full, q_it & 1, abort, p.status))) break;
                 ++q_it;
                 tc_fence_after();
-                {
-                    const int st0 = kv_it % kNS;
-                    if (!(ok = mbar_wait(&bars->k_full[st0], (kv_it / kNS) & 1, abort, p.status))) break;
+                // prologue: S of the first two steps
+                for (int k = 0; k < 2 && k < it.nb && ok; ++k) {
+                    const uint32_t g = kv_it + k;
+                    if (!(ok = mbar_wait(&bars->k_full[g % kNS], (g / kNS) & 1, abort, p.status))) break;
                     tc_fence_after();
-                    const int nk0 = (it.nb >= 2) ? 128 : 64;
                     for (int t = 0; t < it.nt; ++t) {
-                        issue_s(t, st0, nk0);
-                        mma_commit(&bars->s_full[t]);
+                        issue_s(t, g % kNS, k & 1);
+                        mma_commit(&bars->s_full[t][k & 1]);
                     }
-                    if (it.ns == 1) mma_commit(&bars->q_empty);
                 }
-                for (int j = 0; j < it.ns && ok; ++j, ++kv_it) {
+                if (!ok) break;
+                if (it.nb <= 2) mma_commit(&bars->q_empty);
+                for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
                     const int st = kv_it % kNS;
-                    const int nk = (2 * j + 1 < it.nb) ? 128 : 64;
+                    const int buf = k & 1;
                     if (!(ok = mbar_wait(&bars->v_full[st], (kv_it / kNS) & 1, abort, p.status))) break;
                     tc_fence_after();
-                    const bool more = j + 1 < it.ns;
-                    const int st1 = (kv_it + 1) % kNS;
-                    const int nk1 = (2 * (j + 1) + 1 < it.nb) ? 128 : 64;
+                    const bool more = k + 2 < it.nb;
+                    const uint32_t g2 = kv_it + 2;
                     for (int t = 0; t < it.nt && ok; ++t) {
-                        if (!(ok = mbar_wait(&bars->p_full[t], p_it[t] & 1, abort, p.status))) break;
-                        ++p_it[t];
-                        if (j == 0) {
+                        if (!(ok = mbar_wait(&bars->p_full[t][buf], p_it[t][buf] & 1, abort, p.status))) break;
+                        ++p_it[t][buf];
+                        if (k == 0) {
                             if (!(ok = mbar_wait(&bars->o_empty[t], (oe_it[t] & 1) ^ 1, abort, p.status))) break;
                             ++oe_it[t];
                         }
                         tc_fence_after();
-                        issue_pv(t, st, nk, j > 0);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(tmem + 256 * t + 128, tmem + 256 * t + 64 * buf + kk * 8,
+                                   sw128_desc(sKV + st * kStage + kBlk + kk * 2048, kBlkAtom, 1024), id_pv,
+                                   (k > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&bars->o_done[t]);
                         if (more) {
                             if (t == 0) {
-                                if (!(ok = mbar_wait(&bars->k_full[st1], ((kv_it + 1) / kNS) & 1, abort, p.status)))
+                                if (!(ok = mbar_wait(&bars->k_full[g2 % kNS], (g2 / kNS) & 1, abort, p.status)))
                                     break;
                                 tc_fence_after();
                             }
-                            issue_s(t, st1, nk1);
-                            mma_commit(&bars->s_full[t]);
-                        } else {
-                            mma_commit(&bars->o_full[t]);
+                            issue_s(t, g2 % kNS, buf);
+                            mma_commit(&bars->s_full[t][buf]);
                         }
                     }
                     if (!ok) break;
-                    if (j + 2 == it.ns) mma_commit(&bars->q_empty);
+                    if (k + 3 == it.nb) mma_commit(&bars->q_empty);
                     mma_commit(&bars->kv_empty[st]);
                 }
             }
-            // every MMA issued by this thread has finished before TMEM is freed
             mma_commit(&bars->drain);
             volatile int no_abort = 0;
             mbar_wait(&bars->drain, 0, &no_abort, nullptr);
@@ -305,46 +288,54 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int row = quarter * 32 + lane;            // row of the Q tile = TMEM lane
         const int slot_in_tile = row >> 6, r_in = row & 63;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_base + t * 128;
-        const uint32_t tO = tmem + lane_base + 256 + t * 128;
-        uint32_t s_it = 0, o_it = 0;
+        const uint32_t tT = tmem + lane_base + 256 * t;
+        const uint32_t tO = tT + 128;
+        // o_done[t] completes once per PV of this tile; it is waited on phase by
+        // phase (a parity wait is exact only within one phase of the barrier).
+        uint32_t s_it[2] = {0, 0}, pv_it = 0;
         for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
             const Item it = item_of(p, id);
             if (t >= it.nt) continue;
             const int slot = 4 * it.tg + 2 * t + slot_in_tile;
             float m_ref = -INFINITY, l = 0.f;
             bool ok = true;
-            for (int j = 0; j < it.ns; ++j) {
-                const Blk A = block_at(it, 2 * j);
-                const bool hasB = 2 * j + 1 < it.nb;
-                const Blk Bk = hasB ? block_at(it, 2 * j + 1) : A;
-                if (!(ok = mbar_wait(&bars->s_full[t], s_it & 1, abort, p.status))) break;
-                ++s_it;
+            Meta nxt = meta_at(p, it, 0);
+            for (int k = 0; k < it.nb; ++k) {
+                const int buf = k & 1;
+                const Meta m = nxt;
+                if (k + 1 < it.nb) nxt = meta_at(p, it, k + 1);    // prefetch the next block's gate
+                if (!(ok = mbar_wait(&bars->s_full[t][buf], s_it[buf] & 1, abort, p.status))) break;
+                ++s_it[buf];
                 tc_fence_after();
-                // pass 1: row max of the live logits, 32 columns at a time
+                uint32_t raw[2][32];
+                tmem_ld32(tT + 64 * buf, raw[0]);
+                tmem_ld32(tT + 64 * buf + 32, raw[1]);
+                tmem_wait_ld();
+                float x[64];
                 float mx = -INFINITY;
+                if (m.cur || !m.live) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const Blk& bk = q < 2 ? A : Bk;
-                    const bool blk_live = (q < 2 || hasB) && bk.valid;
-                    uint32_t raw[32];
-                    tmem_ld32(tS + q * 32, raw);
-                    tmem_wait_ld();
-                    if (!blk_live) continue;
-                    float bm = -INFINITY;
-                    if (bk.cur) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if ((q & 1) * 32 + e <= r_in) bm = fmaxf(bm, __uint_as_float(raw[e]));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) bm = fmaxf(bm, __uint_as_float(raw[e]));
+                    for (int u = 0; u < 64; ++u) {
+                        const bool live = m.live && u <= r_in;
+                        x[u] = live ? fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2) : -INFINITY;
+                        mx = fmaxf(mx, x[u]);
                     }
-                    if (bm != -INFINITY) mx = fmaxf(mx, fmaf(bm, p.scale2, bk.bias2));
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 64; ++u) {
+                        x[u] = fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2);
+                        mx = fmaxf(mx, x[u]);
+                    }
                 }
                 const float m_new = fmaxf(m_ref, mx);
                 const bool need = m_new > m_ref + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need) && j > 0) {
+                if (k > 0) {
+                    // PV of the previous step is done: O may be rescaled, and the
+                    // o_done phases are observed one by one
+                    if (!(ok = mbar_wait(&bars->o_done[t], (pv_it + k - 1) & 1, abort, p.status))) break;
+                }
+                if (__any_sync(0xffffffffu, need) && k > 0) {
+                    tc_fence_after();
                     const float f = need ? exp2f(m_ref - m_new) : 1.f;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
@@ -361,36 +352,22 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     m_ref = m_new;
                 }
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                // pass 2: P = exp2(logit - m) as bf16 pairs over the consumed S columns
-                // (P columns [16q, 16q+16) lie inside S columns already read)
+                uint32_t pk[32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const Blk& bk = q < 2 ? A : Bk;
-                    const bool blk_live = (q < 2 || hasB) && bk.valid;
-                    uint32_t raw[32];
-                    tmem_ld32(tS + q * 32, raw);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-                    const float off = bk.bias2 - m_use;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int u0 = (q & 1) * 32 + 2 * e;
-                        const bool live0 = blk_live && !(bk.cur && u0 > r_in);
-                        const bool live1 = blk_live && !(bk.cur && u0 + 1 > r_in);
-                        const float p0 = live0 ? exp2f(fmaf(__uint_as_float(raw[2 * e]), p.scale2, off)) : 0.f;
-                        const float p1 = live1 ? exp2f(fmaf(__uint_as_float(raw[2 * e + 1]), p.scale2, off)) : 0.f;
-                        l += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(tS + q * 16, pk);
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = exp2f(x[2 * e] - m_use);
+                    const float p1 = exp2f(x[2 * e + 1] - m_use);
+                    l += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
+                tmem_st32(tT + 64 * buf, pk);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars->p_full[t]);
+                mbar_arrive(&bars->p_full[t][buf]);
             }
             if (!ok) break;
-            if (!mbar_wait(&bars->o_full[t], o_it & 1, abort, p.status)) break;
-            ++o_it;
+            if (!mbar_wait(&bars->o_done[t], (pv_it + it.nb - 1) & 1, abort, p.status)) break;
+            pv_it += it.nb;
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const bool store = slot < p.G;
@@ -429,34 +406,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 }  // namespace
-
-// [rows, H, D] bf16 viewed as 3-D (D, H, rows); 64 x 1 x 64 boxes, 128B swizzle.
-bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    cuuint32_t box[3] = {64, 1, 64};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
 
 cudaError_t launch_fwd_sm100(const AttnArgs& a, void* o, float* lse, cudaStream_t st) {
     CUtensorMap mq, mk, mv;

@@ -205,4 +205,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 }  // namespace sm100
+
+// TMA map of a [rows, H, D] bf16 tensor as 3-D (D, H, rows): 64 x 1 x 64
+// boxes, 128-byte swizzle (tma_maps.cu).
+bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D);
+
 }  // namespace sas

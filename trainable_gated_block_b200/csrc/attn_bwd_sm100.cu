@@ -11,17 +11,21 @@
 //
 // Two tensor-core kernels, no floating-point atomics on dq/dk/dv:
 //  * dq_kernel (query-stationary, like the forward): item = (b, h, i, head
-//    group); per kept block S, dP (tcgen05, SS), dS written back to TMEM as
-//    bf16 and dQ += dS K (tcgen05, A from TMEM); dQ stays in TMEM across the
-//    item. Also the per-block gate gradients.
+//    group), up to two 128-row Q tiles (2 heads x 64 rows each) sharing each
+//    kept K/V block. Per block: S = Q K^T and dP = dO V^T into TMEM, dS to a
+//    swizzled shared-memory tile, dQ += dS K accumulated in TMEM across the
+//    item. Also the per-block gate gradients (warp sums of dS).
 //  * dkv_kernel (key-stationary): item = (b, h, j); walks the query blocks
 //    that attend block j (its own block and every block that kept it, from a
-//    reverse index), all query heads of the group, and accumulates
-//    dV^T = sum dO^T P and dK^T = sum Q^T dS in TMEM (M = head dim).
-// The cost is two recomputations of S and dP instead of one; in exchange
+//    reverse index), one Q tile per step, and accumulates dV^T = sum dO^T P
+//    and dK^T = sum Q^T dS in TMEM (M = head dim).
+// S and dP are computed twice (once per kernel) instead of once; in exchange
 // nothing is reduced through global memory and dq/dk/dv are deterministic.
-#include <cudaTypedefs.h>
-
+//
+// Barrier discipline: every mbarrier phase is waited on in order by its
+// consumer (a parity wait is exact only within one phase of the barrier), so
+// "buffer is free again" barriers are waited on before every reuse of the
+// buffer except the first.
 #include "launch.h"
 #include "sm100.cuh"
 
@@ -37,6 +41,7 @@ constexpr uint32_t kTileAtom = 2 * kBox;   // 128 rows x 128 B (one 64-column ha
 constexpr uint32_t kTile = 2 * kTileAtom;  // 128 rows x 256 B
 constexpr uint32_t kBlkAtom = kBox;        // 64 keys x 128 B
 constexpr uint32_t kBlk = 2 * kBlkAtom;    // 64 keys x 256 B
+constexpr uint32_t kRowTile = 128 * 128;   // 128 rows x 64 bf16 (P or dS of one Q tile)
 
 // ------------------------------------------------------------------ shared
 struct Params {
@@ -57,21 +62,29 @@ struct Params {
     int* status;
 };
 
+// Writes 64 bf16 pairs-packed values (one 128-byte row) into a 128B-swizzled tile.
+__device__ __forceinline__ void store_row(uint8_t* tile, int row, const uint32_t (&v)[32]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(tile + sw128_offset(row, c)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
 // ===================================================================== dq
 namespace dqk {
 
-constexpr uint32_t kOffQ = 0;                      // 2 tiles
-constexpr uint32_t kOffO = 2 * kTile;              // dO, 2 tiles
+constexpr uint32_t kOffQ = 0;                      // 2 Q tiles
+constexpr uint32_t kOffO = 2 * kTile;              // 2 dO tiles
 constexpr uint32_t kOffKV = 4 * kTile;             // 2 stages x (K block, V block)
 constexpr int kNS = 2;
 constexpr uint32_t kStage = 2 * kBlk;
-constexpr uint32_t kOffBar = kOffKV + kNS * kStage;   // 192 KB
+constexpr uint32_t kOffDS = kOffKV + kNS * kStage;        // 2 dS tiles
+constexpr uint32_t kOffBar = kOffDS + 2 * kRowTile;      // 224 KB
 constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
 
 struct Bars {
     uint64_t qd_full, qd_empty;
     uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
-    uint64_t s_full[2], ds_full[2], dq_full[2], dq_empty[2];
+    uint64_t s_full[2], tm_free[2], ds_full[2], ds_empty[2], dq_full[2], dq_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -138,7 +151,9 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->tm_free[t], 128);
             mbar_init(&bars->ds_full[t], 128);
+            mbar_init(&bars->ds_empty[t], 1);
             mbar_init(&bars->dq_full[t], 1);
             mbar_init(&bars->dq_empty[t], 128);
         }
@@ -155,6 +170,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const uint32_t sQ = smem_u32(smem + kOffQ), sO = smem_u32(smem + kOffO), sKV = smem_u32(smem + kOffKV);
+    const uint32_t sDS = smem_u32(smem + kOffDS);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -208,8 +224,13 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_dq = idesc_bf16(128, kD, false, true);
-            uint32_t kv_it = 0, q_it = 0, ds_it[2] = {0, 0}, de_it[2] = {0, 0};
-            auto issue_sdp = [&](int t, int st) {
+            uint32_t kv_it = 0, q_it = 0, ds_it[2] = {0, 0}, de_it[2] = {0, 0}, sdp_n[2] = {0, 0};
+            bool ok = true;
+            // S and dP of tile t for the block in stage st, once its TMEM columns are free
+            auto issue_sdp = [&](int t, int st) -> bool {
+                if (sdp_n[t] > 0 && !mbar_wait(&bars->tm_free[t], (sdp_n[t] - 1) & 1, abort, p.status)) return false;
+                ++sdp_n[t];
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t ao = t * kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
@@ -223,8 +244,9 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     mma_ss(tmem + 256 * t + 64, sw128_desc(sO + ao, 16, 1024), sw128_desc(sKV + bo, 16, 1024), id_s,
                            kk > 0);
                 }
+                mma_commit(&bars->s_full[t]);
+                return true;
             };
-            bool ok = true;
             for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
                 const Item it = item_of(p, id);
                 if (!(ok = mbar_wait(&bars->qd_full, q_it & 1, abort, p.status))) break;
@@ -234,19 +256,21 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     const uint32_t ph = (kv_it / kNS) & 1;
                     if (!(ok = mbar_wait(&bars->k_full[st0], ph, abort, p.status))) break;
                     if (!(ok = mbar_wait(&bars->v_full[st0], ph, abort, p.status))) break;
-                    tc_fence_after();
-                    for (int t = 0; t < it.nt; ++t) {
-                        issue_sdp(t, st0);
-                        mma_commit(&bars->s_full[t]);
-                    }
+                    for (int t = 0; t < it.nt && ok; ++t) ok = issue_sdp(t, st0);
+                    if (!ok) break;
                     if (it.nb == 1) mma_commit(&bars->qd_empty);
                 }
                 for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
                     const int st = kv_it % kNS;
                     const bool more = k + 1 < it.nb;
-                    const int st1 = (kv_it + 1) % kNS;
-                    const uint32_t ph1 = ((kv_it + 1) / kNS) & 1;
+                    if (more) {
+                        const int st1 = (kv_it + 1) % kNS;
+                        const uint32_t ph1 = ((kv_it + 1) / kNS) & 1;
+                        if (!(ok = mbar_wait(&bars->k_full[st1], ph1, abort, p.status))) break;
+                        if (!(ok = mbar_wait(&bars->v_full[st1], ph1, abort, p.status))) break;
+                    }
                     for (int t = 0; t < it.nt && ok; ++t) {
+                        if (more && !(ok = issue_sdp(t, (kv_it + 1) % kNS))) break;
                         if (!(ok = mbar_wait(&bars->ds_full[t], ds_it[t] & 1, abort, p.status))) break;
                         ++ds_it[t];
                         if (k == 0) {
@@ -256,20 +280,11 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + 256 * t + 128, tmem + 256 * t + kk * 8,
+                            mma_ss(tmem + 256 * t + 128, sw128_desc(sDS + t * kRowTile + kk * 32, 16, 1024),
                                    sw128_desc(sKV + st * kStage + kk * 2048, kBlkAtom, 1024), id_dq,
                                    (k > 0 || kk > 0) ? 1u : 0u);
-                        if (more) {
-                            if (t == 0) {
-                                if (!(ok = mbar_wait(&bars->k_full[st1], ph1, abort, p.status))) break;
-                                if (!(ok = mbar_wait(&bars->v_full[st1], ph1, abort, p.status))) break;
-                                tc_fence_after();
-                            }
-                            issue_sdp(t, st1);
-                            mma_commit(&bars->s_full[t]);
-                        } else {
-                            mma_commit(&bars->dq_full[t]);
-                        }
+                        mma_commit(&bars->ds_empty[t]);
+                        if (!more) mma_commit(&bars->dq_full[t]);
                     }
                     if (!ok) break;
                     if (k + 2 == it.nb) mma_commit(&bars->qd_empty);
@@ -289,7 +304,8 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
         const uint32_t tS = tmem + lane_base + 256 * t;
         const uint32_t tP = tS + 64;
         const uint32_t tQ = tS + 128;
-        uint32_t s_it = 0, q_it = 0;
+        uint8_t* ds_tile = smem + kOffDS + t * kRowTile;
+        uint32_t s_it = 0, q_it = 0, ds_n = 0;
         for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
             const Item it = item_of(p, id);
             if (t >= it.nt) continue;
@@ -300,39 +316,50 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             const float lse2 = p.lse[lrow] * kLog2e;
             const float drow = p.Dr[lrow];
             bool ok = true;
+            Blk nxt = block_at(p, it, 0);
             for (int k = 0; k < it.nb; ++k) {
-                const Blk bk = block_at(p, it, k);
+                const Blk bk = nxt;
+                if (k + 1 < it.nb) nxt = block_at(p, it, k + 1);
                 if (!(ok = mbar_wait(&bars->s_full[t], s_it & 1, abort, p.status))) break;
                 ++s_it;
                 tc_fence_after();
-                uint32_t sv[2][32], pv[2][32];
-                tmem_ld32(tS, sv[0]);
-                tmem_ld32(tS + 32, sv[1]);
-                tmem_ld32(tP, pv[0]);
-                tmem_ld32(tP + 32, pv[1]);
-                tmem_wait_ld();
                 const float off = bk.bias2 - lse2;
                 float gs = 0.f;
-                uint32_t pk[32];
+                // dQ of the previous step has finished reading the dS tile
+                if (ds_n > 0 && !(ok = mbar_wait(&bars->ds_empty[t], (ds_n - 1) & 1, abort, p.status))) break;
+                ++ds_n;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float d2[2];
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int u = 2 * e + q;
-                        const bool live = row_ok && bk.valid && !(bk.cur && u > r_in);
-                        const float s = __uint_as_float(sv[u >> 5][u & 31]);
-                        const float dp = __uint_as_float(pv[u >> 5][u & 31]);
-                        const float pr = live ? exp2f(fmaf(s, p.scale2, off)) : 0.f;
-                        const float ds = pr * (dp - drow);
-                        gs += ds;
-                        d2[q] = ds * p.sm_scale;
+                for (int hf = 0; hf < 2; ++hf) {          // keys [32 hf, 32 hf + 32)
+                    uint32_t sv[32], pv[32];
+                    tmem_ld32(tS + 32 * hf, sv);
+                    tmem_ld32(tP + 32 * hf, pv);
+                    tmem_wait_ld();
+                    if (hf == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&bars->tm_free[t]);   // S/dP columns may be refilled
                     }
-                    pk[e] = pack_bf16x2(d2[0], d2[1]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {         // 16-byte chunk = keys 8c .. 8c+7 of the half
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float d2[2];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int e = 8 * c + 2 * e2 + q;
+                                const bool live = row_ok && bk.valid && !(bk.cur && 32 * hf + e > r_in);
+                                const float pr = live ? exp2f(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
+                                const float ds = pr * (__uint_as_float(pv[e]) - drow);
+                                gs += ds;
+                                d2[q] = ds * p.sm_scale;
+                            }
+                            pk[e2] = pack_bf16x2(d2[0], d2[1]);
+                        }
+                        *reinterpret_cast<uint4*>(ds_tile + sw128_offset(row, 4 * hf + c)) =
+                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
                 }
-                tmem_st32(tS, pk);
-                tmem_wait_st();
-                tc_fence_before();
+                fence_proxy_async_smem();
                 mbar_arrive(&bars->ds_full[t]);
                 if (!bk.cur && bk.valid) {
                     gs = warp_sum(gs);
@@ -384,15 +411,14 @@ constexpr uint32_t kOffV = kBlk;                   // V_j
 constexpr uint32_t kOffStage = 2 * kBlk;           // 2 stages x (Q tile, dO tile)
 constexpr int kNS = 2;
 constexpr uint32_t kStage = 2 * kTile;
-constexpr uint32_t kOffPS = kOffStage + kNS * kStage;    // per warpgroup: P (128 x 64 bf16), dS
-constexpr uint32_t kPSBuf = 128 * 128;                    // 16 KB
-constexpr uint32_t kOffBar = kOffPS + 2 * 2 * kPSBuf;     // 224 KB
+constexpr uint32_t kOffPS = kOffStage + kNS * kStage;    // per warpgroup: P tile, dS tile
+constexpr uint32_t kOffBar = kOffPS + 2 * 2 * kRowTile;  // 224 KB
 constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
 
 struct Bars {
     uint64_t kv_full, kv_empty;
     uint64_t qd_full[kNS], qd_empty[kNS];
-    uint64_t s_full[2], pds_full[2], pds_empty[2];
+    uint64_t s_full[2], tm_free[2], pds_full[2], pds_empty[2];
     uint64_t acc_full, acc_empty;
     uint64_t drain;
     uint32_t tmem_base;
@@ -412,6 +438,39 @@ __device__ __forceinline__ int n_entries(const Params& p, long long bh, int j) {
     return max(1, min(n, p.NQB - j));
 }
 
+// What a softmax thread needs for step m of item (b, h, j): the query block,
+// the gate of block j in that block's selection, and its row's LSE and Dr.
+struct StepMeta {
+    int i;
+    bool cur, row_ok;
+    float bias2, lse2, drow;
+};
+__device__ __forceinline__ StepMeta step_meta(const Params& p, const int32_t* list, int b, int h, long long bh, int j,
+                                              int m, int row) {
+    StepMeta s;
+    const int e = m / p.ntile, t = m % p.ntile;
+    const int ent = __ldg(list + e);
+    int i = ent >> 16;
+    const int slot = ent & 0xFFFF;
+    bool valid = i >= j && i < p.NQB;
+    if (!valid) i = j;
+    s.i = i;
+    s.cur = (i == j);
+    s.bias2 = 0.f;
+    if (!s.cur) {
+        const long long srow = bh * p.NQB + i;
+        valid = valid && slot < p.K && __ldg(p.idx + srow * p.K + slot) == j;
+        s.bias2 = valid ? __ldg(p.log_gate + srow * p.K + slot) * kLog2e : 0.f;
+    }
+    const int hs = 2 * t + (row >> 6);
+    s.row_ok = valid && hs < p.G;
+    const int hq = h * p.G + (hs < p.G ? hs : 0);
+    const long long lrow = ((long long)b * p.Hq + hq) * p.S + (long long)i * 64 + (row & 63);
+    s.lse2 = __ldg(p.lse + lrow) * kLog2e;
+    s.drow = __ldg(p.Dr + lrow);
+    return s;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
            const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const Params p) {
@@ -429,6 +488,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         }
         for (int w = 0; w < 2; ++w) {
             mbar_init(&bars->s_full[w], 1);
+            mbar_init(&bars->tm_free[w], 128);
             mbar_init(&bars->pds_full[w], 128);
             mbar_init(&bars->pds_empty[w], 1);
         }
@@ -502,9 +562,9 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_t = idesc_bf16(128, 64, true, true);
-            uint32_t item_it = 0, qd_it = 0, pds_it[2] = {0, 0};
+            uint32_t item_it = 0, qd_it = 0, pds_it[2] = {0, 0}, sdp_n[2] = {0, 0};
             bool ok = true;
-            // dV^T += dO^T P, dK^T += Q^T dS for step m (stage st, warpgroup w)
+            // dV^T += dO^T P, dK^T += Q^T dS for step m (stage st, warpgroup m & 1)
             auto dvdk = [&](int m, int st, uint32_t item_parity) -> bool {
                 const int w = m & 1;
                 if (!mbar_wait(&bars->pds_full[w], pds_it[w] & 1, abort, p.status)) return false;
@@ -512,15 +572,15 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (m == 0 && !mbar_wait(&bars->acc_empty, item_parity ^ 1, abort, p.status)) return false;
                 tc_fence_after();
                 const uint32_t sq = s_base + kOffStage + st * kStage;
-                const uint32_t sp = s_base + kOffPS + w * 2 * kPSBuf;
+                const uint32_t sp = s_base + kOffPS + w * 2 * kRowTile;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem + 256, sw128_desc(sq + kTile + kk * 2048, kTileAtom, 1024),
-                           sw128_desc(sp + kk * 2048, kPSBuf, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
+                           sw128_desc(sp + kk * 2048, kRowTile, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem + 320, sw128_desc(sq + kk * 2048, kTileAtom, 1024),
-                           sw128_desc(sp + kPSBuf + kk * 2048, kPSBuf, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
+                           sw128_desc(sp + kRowTile + kk * 2048, kRowTile, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bars->qd_empty[st]);
                 mma_commit(&bars->pds_empty[w]);
                 return true;
@@ -537,6 +597,10 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                     const int st = qd_it % kNS;
                     const int w = m & 1;
                     if (!(ok = mbar_wait(&bars->qd_full[st], (qd_it / kNS) & 1, abort, p.status))) break;
+                    // this warpgroup has loaded its previous S/dP out of TMEM
+                    if (sdp_n[w] > 0 && !(ok = mbar_wait(&bars->tm_free[w], (sdp_n[w] - 1) & 1, abort, p.status)))
+                        break;
+                    ++sdp_n[w];
                     tc_fence_after();
                     const uint32_t sq = s_base + kOffStage + st * kStage;
 #pragma unroll
@@ -573,9 +637,9 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         const int r_in = row & 63;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_base + 128 * w;
-        uint8_t* bufP = smem + kOffPS + w * 2 * kPSBuf;
-        uint8_t* bufS = bufP + kPSBuf;
-        uint32_t s_it = 0, pe_it = 0, item_it = 0;
+        uint8_t* bufP = smem + kOffPS + w * 2 * kRowTile;
+        uint8_t* bufS = bufP + kRowTile;
+        uint32_t s_it = 0, pds_n = 0, item_it = 0;
         bool ok = true;
         for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
             int b, h, j;
@@ -583,63 +647,50 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             item_of(p, id, b, h, j, bh);
             const int N = n_entries(p, bh, j) * p.ntile;
             const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
+            StepMeta nxt;
+            if (w < N) nxt = step_meta(p, list, b, h, bh, j, w, row);
             for (int m = w; m < N; m += 2) {
-                const int e = m / p.ntile, t = m % p.ntile;
-                const int ent = __ldg(list + e);
-                int i = ent >> 16;
-                const int slot = ent & 0xFFFF;
-                bool valid = i >= j && i < p.NQB;
-                if (!valid) i = j;
-                const bool cur = (i == j);
-                float bias2 = 0.f;
-                if (!cur) {
-                    const long long srow = bh * p.NQB + i;
-                    valid = valid && slot < p.K && __ldg(p.idx + srow * p.K + slot) == j;
-                    bias2 = valid ? __ldg(p.log_gate + srow * p.K + slot) * kLog2e : 0.f;
-                }
-                const int hs = 2 * t + (row >> 6);
-                const bool row_ok = valid && hs < p.G;
-                const int hq = h * p.G + (hs < p.G ? hs : 0);
-                const long long lrow = ((long long)b * p.Hq + hq) * p.S + (long long)i * 64 + r_in;
-                const float lse2 = p.lse[lrow] * kLog2e;
-                const float drow = p.Dr[lrow];
+                const StepMeta sm = nxt;
+                if (m + 2 < N) nxt = step_meta(p, list, b, h, bh, j, m + 2, row);   // prefetch
                 if (!(ok = mbar_wait(&bars->s_full[w], s_it & 1, abort, p.status))) break;
                 ++s_it;
                 tc_fence_after();
+                const float off = sm.bias2 - sm.lse2;
                 // the MMA of this warpgroup's previous step has finished reading the buffers
-                if (!(ok = mbar_wait(&bars->pds_empty[w], (pe_it & 1) ^ 1, abort, p.status))) break;
-                ++pe_it;
-                const float off = bias2 - lse2;
+                if (pds_n > 0 && !(ok = mbar_wait(&bars->pds_empty[w], (pds_n - 1) & 1, abort, p.status))) break;
+                ++pds_n;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {           // keys [32 hf, 32 hf + 32)
+                for (int hf = 0; hf < 2; ++hf) {          // keys [32 hf, 32 hf + 32)
                     uint32_t sv[32], pv[32];
                     tmem_ld32(tS + 32 * hf, sv);
                     tmem_ld32(tS + 64 + 32 * hf, pv);
                     tmem_wait_ld();
-                    uint32_t pp[16], dd[16];
-#pragma unroll
-                    for (int e2 = 0; e2 < 16; ++e2) {
-                        float pr2[2], ds2[2];
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const int u = 32 * hf + 2 * e2 + q;
-                            const bool live = row_ok && !(cur && u > r_in);
-                            pr2[q] = live ? exp2f(fmaf(__uint_as_float(sv[2 * e2 + q]), p.scale2, off)) : 0.f;
-                            ds2[q] = pr2[q] * (__uint_as_float(pv[2 * e2 + q]) - drow) * p.sm_scale;
-                        }
-                        pp[e2] = pack_bf16x2(pr2[0], pr2[1]);
-                        dd[e2] = pack_bf16x2(ds2[0], ds2[1]);
+                    if (hf == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&bars->tm_free[w]);   // S/dP columns may be refilled
                     }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        *reinterpret_cast<uint4*>(bufP + sw128_offset(row, 4 * hf + c)) =
-                            make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
-                        *reinterpret_cast<uint4*>(bufS + sw128_offset(row, 4 * hf + c)) =
-                            make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+                    for (int c = 0; c < 4; ++c) {         // 16-byte chunk = keys 8c .. 8c+7 of the half
+                        uint32_t pp[4], dd[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float pr2[2], ds2[2];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int e = 8 * c + 2 * e2 + q;
+                                const bool live = sm.row_ok && !(sm.cur && 32 * hf + e > r_in);
+                                pr2[q] = live ? exp2f(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
+                                ds2[q] = pr2[q] * (__uint_as_float(pv[e]) - sm.drow) * p.sm_scale;
+                            }
+                            pp[e2] = pack_bf16x2(pr2[0], pr2[1]);
+                            dd[e2] = pack_bf16x2(ds2[0], ds2[1]);
+                        }
+                        const int ch = 4 * hf + c;
+                        *reinterpret_cast<uint4*>(bufP + sw128_offset(row, ch)) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
+                        *reinterpret_cast<uint4*>(bufS + sw128_offset(row, ch)) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
                     }
                 }
                 fence_proxy_async_smem();
-                tc_fence_before();
                 mbar_arrive(&bars->pds_full[w]);
             }
             if (!ok) break;

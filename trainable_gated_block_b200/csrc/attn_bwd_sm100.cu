@@ -35,13 +35,17 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 two warpgroups
+// warp 0 TMA, warps 1 and 10 MMA issuers (one thread each: a single thread
+// issues tcgen05.mma at a bounded rate), warps 2-5 / 6-9 two warpgroups
+constexpr int kThreads = 352;
+constexpr int kIssuer1Warp = 10;
 constexpr uint32_t kBox = 64 * 128;        // TMA box: 64 rows x 128 B
 constexpr uint32_t kTileAtom = 2 * kBox;   // 128 rows x 128 B (one 64-column half of a Q/dO tile)
 constexpr uint32_t kTile = 2 * kTileAtom;  // 128 rows x 256 B
 constexpr uint32_t kBlkAtom = kBox;        // 64 keys x 128 B
 constexpr uint32_t kBlk = 2 * kBlkAtom;    // 64 keys x 256 B
 constexpr uint32_t kRowTile = 128 * 128;   // 128 rows x 64 bf16 (P or dS of one Q tile)
+constexpr uint32_t kHi = sm100::sdesc_hi(1024);   // high descriptor word: 8-row groups 1024 B apart
 
 // ------------------------------------------------------------------ shared
 struct Params {
@@ -85,7 +89,7 @@ struct Bars {
     uint64_t qd_full, qd_empty;
     uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
     uint64_t s_full[2], tm_free[2], ds_full[2], ds_empty[2], dq_full[2], dq_empty[2];
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -143,11 +147,11 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
     volatile int* abort = &bars->abort;
     if (threadIdx.x == 0) {
         mbar_init(&bars->qd_full, 1);
-        mbar_init(&bars->qd_empty, 1);
+        mbar_init(&bars->qd_empty, 2);                  // one arrival per MMA issuer
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
+            mbar_init(&bars->kv_empty[s], 2);
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars->s_full[t], 1);
@@ -156,8 +160,8 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             mbar_init(&bars->ds_empty[t], 1);
             mbar_init(&bars->dq_full[t], 1);
             mbar_init(&bars->dq_empty[t], 128);
+            mbar_init(&bars->drain[t], 1);
         }
-        mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -220,35 +224,43 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                 if (q_issued) mbar_wait(&bars->qd_full, (q_it - 1) & 1, &no_abort, nullptr);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kIssuer1Warp) {
         if (lane == 0) {
+            const int t = (warp == 1) ? 0 : 1;          // the Q tile this thread issues for
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_dq = idesc_bf16(128, kD, false, true);
-            uint32_t kv_it = 0, q_it = 0, ds_it[2] = {0, 0}, de_it[2] = {0, 0}, sdp_n[2] = {0, 0};
+            uint32_t kv_it = 0, q_it = 0, ds_it = 0, de_it = 0, sdp_n = 0;
             bool ok = true;
-            // S and dP of tile t for the block in stage st, once its TMEM columns are free
-            auto issue_sdp = [&](int t, int st) -> bool {
-                if (sdp_n[t] > 0 && !mbar_wait(&bars->tm_free[t], (sdp_n[t] - 1) & 1, abort, p.status)) return false;
-                ++sdp_n[t];
+            const uint32_t q_lo = sdesc_lo(sQ + t * kTile, 16), o_lo = sdesc_lo(sO + t * kTile, 16);
+            // S and dP of this tile for the block in stage st, once its TMEM columns are free
+            auto issue_sdp = [&](int st) -> bool {
+                if (sdp_n > 0 && !mbar_wait(&bars->tm_free[t], (sdp_n - 1) & 1, abort, p.status)) return false;
+                ++sdp_n;
                 tc_fence_after();
+                const uint32_t kv_lo = sdesc_lo(sKV + st * kStage, 16);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t ao = t * kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                    const uint32_t bo = st * kStage + (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                    mma_ss(tmem + 256 * t, sw128_desc(sQ + ao, 16, 1024), sw128_desc(sKV + bo, 16, 1024), id_s, kk > 0);
+                    const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                    mma_ss_w(tmem + 256 * t, q_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi, id_s, kk > 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t ao = t * kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                    const uint32_t bo = st * kStage + kBlk + (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                    mma_ss(tmem + 256 * t + 64, sw128_desc(sO + ao, 16, 1024), sw128_desc(sKV + bo, 16, 1024), id_s,
-                           kk > 0);
+                    const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                    const uint32_t bo = kBlk + (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                    mma_ss_w(tmem + 256 * t + 64, o_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi, id_s, kk > 0);
                 }
                 mma_commit(&bars->s_full[t]);
                 return true;
             };
             for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
                 const Item it = item_of(p, id);
+                if (t >= it.nt) {                       // tile 1 idle: tile 0's issuer arrives for it
+                    kv_it += it.nb;
+                    ++q_it;
+                    continue;
+                }
+                const int owe = (it.nt == 1) ? 2 : 1;   // arrivals owed to the shared stage barriers
                 if (!(ok = mbar_wait(&bars->qd_full, q_it & 1, abort, p.status))) break;
                 ++q_it;
                 {
@@ -256,9 +268,9 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     const uint32_t ph = (kv_it / kNS) & 1;
                     if (!(ok = mbar_wait(&bars->k_full[st0], ph, abort, p.status))) break;
                     if (!(ok = mbar_wait(&bars->v_full[st0], ph, abort, p.status))) break;
-                    for (int t = 0; t < it.nt && ok; ++t) ok = issue_sdp(t, st0);
-                    if (!ok) break;
-                    if (it.nb == 1) mma_commit(&bars->qd_empty);
+                    if (!(ok = issue_sdp(st0))) break;
+                    if (it.nb == 1)
+                        for (int c = 0; c < owe; ++c) mma_commit(&bars->qd_empty);
                 }
                 for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
                     const int st = kv_it % kNS;
@@ -268,34 +280,34 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                         const uint32_t ph1 = ((kv_it + 1) / kNS) & 1;
                         if (!(ok = mbar_wait(&bars->k_full[st1], ph1, abort, p.status))) break;
                         if (!(ok = mbar_wait(&bars->v_full[st1], ph1, abort, p.status))) break;
+                        if (!(ok = issue_sdp(st1))) break;
                     }
-                    for (int t = 0; t < it.nt && ok; ++t) {
-                        if (more && !(ok = issue_sdp(t, (kv_it + 1) % kNS))) break;
-                        if (!(ok = mbar_wait(&bars->ds_full[t], ds_it[t] & 1, abort, p.status))) break;
-                        ++ds_it[t];
-                        if (k == 0) {
-                            if (!(ok = mbar_wait(&bars->dq_empty[t], (de_it[t] & 1) ^ 1, abort, p.status))) break;
-                            ++de_it[t];
-                        }
-                        tc_fence_after();
+                    if (!(ok = mbar_wait(&bars->ds_full[t], ds_it & 1, abort, p.status))) break;
+                    ++ds_it;
+                    if (k == 0) {
+                        if (!(ok = mbar_wait(&bars->dq_empty[t], (de_it & 1) ^ 1, abort, p.status))) break;
+                        ++de_it;
+                    }
+                    tc_fence_after();
+                    const uint32_t ds_lo = sdesc_lo(sDS + t * kRowTile, 16);         // K-major dS
+                    const uint32_t kt_lo = sdesc_lo(sKV + st * kStage, kBlkAtom);    // MN-major K
+                    const uint32_t acc0 = k > 0 ? 1u : 0u;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(tmem + 256 * t + 128, sw128_desc(sDS + t * kRowTile + kk * 32, 16, 1024),
-                                   sw128_desc(sKV + st * kStage + kk * 2048, kBlkAtom, 1024), id_dq,
-                                   (k > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&bars->ds_empty[t]);
-                        if (!more) mma_commit(&bars->dq_full[t]);
-                    }
-                    if (!ok) break;
-                    if (k + 2 == it.nb) mma_commit(&bars->qd_empty);
-                    mma_commit(&bars->kv_empty[st]);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss_w(tmem + 256 * t + 128, ds_lo + ((kk * 32) >> 4), kHi, kt_lo + ((kk * 2048) >> 4), kHi,
+                                 id_dq, kk > 0 ? 1u : acc0);
+                    mma_commit(&bars->ds_empty[t]);
+                    if (!more) mma_commit(&bars->dq_full[t]);
+                    if (k + 2 == it.nb)
+                        for (int c = 0; c < owe; ++c) mma_commit(&bars->qd_empty);
+                    for (int c = 0; c < owe; ++c) mma_commit(&bars->kv_empty[st]);
                 }
             }
-            mma_commit(&bars->drain);
+            mma_commit(&bars->drain[t]);
             volatile int no_abort = 0;
-            mbar_wait(&bars->drain, 0, &no_abort, nullptr);
+            mbar_wait(&bars->drain[t], 0, &no_abort, nullptr);
         }
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         const int t = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
@@ -420,7 +432,7 @@ struct Bars {
     uint64_t qd_full[kNS], qd_empty[kNS];
     uint64_t s_full[2], tm_free[2], pds_full[2], pds_empty[2];
     uint64_t acc_full, acc_empty;
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -481,7 +493,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     volatile int* abort = &bars->abort;
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
-        mbar_init(&bars->kv_empty, 1);
+        mbar_init(&bars->kv_empty, 2);                  // one arrival per MMA issuer
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&bars->qd_full[s], 1);
             mbar_init(&bars->qd_empty[s], 1);
@@ -491,10 +503,10 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             mbar_init(&bars->tm_free[w], 128);
             mbar_init(&bars->pds_full[w], 128);
             mbar_init(&bars->pds_empty[w], 1);
+            mbar_init(&bars->drain[w], 1);
         }
-        mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->acc_full, 2);
         mbar_init(&bars->acc_empty, 256);
-        mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -558,79 +570,76 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (kv_issued) mbar_wait(&bars->kv_full, (item_it - 1) & 1, &no_abort, nullptr);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kIssuer1Warp) {
+        // one issuer per warpgroup: issuer w runs the steps m = w, w+2, ... of each
+        // item and accumulates its own dV^T, dK^T (the drain adds the two)
         if (lane == 0) {
+            const int w = (warp == 1) ? 0 : 1;
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_t = idesc_bf16(128, 64, true, true);
-            uint32_t item_it = 0, qd_it = 0, pds_it[2] = {0, 0}, sdp_n[2] = {0, 0};
+            const uint32_t k_lo = sdesc_lo(s_base + kOffK, 16), v_lo = sdesc_lo(s_base + kOffV, 16);
+            const uint32_t plo = sdesc_lo(s_base + kOffPS + w * 2 * kRowTile, kRowTile);   // P, dS (MN-major)
+            const uint32_t acc_v = tmem + 256 + 128 * w, acc_k = acc_v + 64;
+            uint32_t item_it = 0, gbase = 0, pds_it = 0, sdp_n = 0;
             bool ok = true;
-            // dV^T += dO^T P, dK^T += Q^T dS for step m (stage st, warpgroup m & 1)
-            auto dvdk = [&](int m, int st, uint32_t item_parity) -> bool {
-                const int w = m & 1;
-                if (!mbar_wait(&bars->pds_full[w], pds_it[w] & 1, abort, p.status)) return false;
-                ++pds_it[w];
-                if (m == 0 && !mbar_wait(&bars->acc_empty, item_parity ^ 1, abort, p.status)) return false;
-                tc_fence_after();
-                const uint32_t sq = s_base + kOffStage + st * kStage;
-                const uint32_t sp = s_base + kOffPS + w * 2 * kRowTile;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + 256, sw128_desc(sq + kTile + kk * 2048, kTileAtom, 1024),
-                           sw128_desc(sp + kk * 2048, kRowTile, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + 320, sw128_desc(sq + kk * 2048, kTileAtom, 1024),
-                           sw128_desc(sp + kRowTile + kk * 2048, kRowTile, 1024), id_t, (m > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&bars->qd_empty[st]);
-                mma_commit(&bars->pds_empty[w]);
-                return true;
-            };
             for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
                 int b, h, j;
                 long long bh;
                 item_of(p, id, b, h, j, bh);
                 const int N = n_entries(p, bh, j) * p.ntile;
                 if (!(ok = mbar_wait(&bars->kv_full, item_it & 1, abort, p.status))) break;
+                // the drain of the previous item has read both accumulators
+                if (!(ok = mbar_wait(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
                 tc_fence_after();
-                int prev_st = 0;
-                for (int m = 0; m < N && ok; ++m, ++qd_it) {
-                    const int st = qd_it % kNS;
-                    const int w = m & 1;
-                    if (!(ok = mbar_wait(&bars->qd_full[st], (qd_it / kNS) & 1, abort, p.status))) break;
+                for (int m = w; m < N && ok; m += 2) {
+                    const uint32_t g = gbase + m;
+                    const int st = g % kNS;
+                    if (!(ok = mbar_wait(&bars->qd_full[st], (g / kNS) & 1, abort, p.status))) break;
                     // this warpgroup has loaded its previous S/dP out of TMEM
-                    if (sdp_n[w] > 0 && !(ok = mbar_wait(&bars->tm_free[w], (sdp_n[w] - 1) & 1, abort, p.status)))
-                        break;
-                    ++sdp_n[w];
+                    if (sdp_n > 0 && !(ok = mbar_wait(&bars->tm_free[w], (sdp_n - 1) & 1, abort, p.status))) break;
+                    ++sdp_n;
                     tc_fence_after();
-                    const uint32_t sq = s_base + kOffStage + st * kStage;
+                    const uint32_t qk = sdesc_lo(s_base + kOffStage + st * kStage, 16);   // K-major Q, dO
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
                         const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                        mma_ss(tmem + 128 * w, sw128_desc(sq + ao, 16, 1024), sw128_desc(s_base + kOffK + bo, 16, 1024),
-                               id_s, kk > 0);
+                        mma_ss_w(tmem + 128 * w, qk + (ao >> 4), kHi, k_lo + (bo >> 4), kHi, id_s, kk > 0);
                     }
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t ao = kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
                         const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                        mma_ss(tmem + 128 * w + 64, sw128_desc(sq + ao, 16, 1024),
-                               sw128_desc(s_base + kOffV + bo, 16, 1024), id_s, kk > 0);
+                        mma_ss_w(tmem + 128 * w + 64, qk + (ao >> 4), kHi, v_lo + (bo >> 4), kHi, id_s, kk > 0);
                     }
                     mma_commit(&bars->s_full[w]);
-                    if (m > 0 && !(ok = dvdk(m - 1, prev_st, item_it & 1))) break;
-                    prev_st = st;
+                    // dV^T += dO^T P, dK^T += Q^T dS once the warpgroup wrote P and dS
+                    if (!(ok = mbar_wait(&bars->pds_full[w], pds_it & 1, abort, p.status))) break;
+                    ++pds_it;
+                    tc_fence_after();
+                    const uint32_t qlo = sdesc_lo(s_base + kOffStage + st * kStage, kTileAtom);   // MN-major Q, dO
+                    const uint32_t acc0 = (m >= 2) ? 1u : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss_w(acc_v, qlo + ((kTile + kk * 2048) >> 4), kHi, plo + ((kk * 2048) >> 4), kHi, id_t,
+                                 kk > 0 ? 1u : acc0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss_w(acc_k, qlo + ((kk * 2048) >> 4), kHi, plo + ((kRowTile + kk * 2048) >> 4), kHi, id_t,
+                                 kk > 0 ? 1u : acc0);
+                    mma_commit(&bars->qd_empty[st]);
+                    mma_commit(&bars->pds_empty[w]);
                 }
                 if (!ok) break;
-                if (!(ok = dvdk(N - 1, prev_st, item_it & 1))) break;
+                gbase += N;
                 mma_commit(&bars->kv_empty);
                 mma_commit(&bars->acc_full);
             }
-            mma_commit(&bars->drain);
+            mma_commit(&bars->drain[w]);
             volatile int no_abort = 0;
-            mbar_wait(&bars->drain, 0, &no_abort, nullptr);
+            mbar_wait(&bars->drain[w], 0, &no_abort, nullptr);
         }
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         const int w = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
@@ -694,7 +703,9 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 mbar_arrive(&bars->pds_full[w]);
             }
             if (!ok) break;
-            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim index)
+            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim
+            // index); each is the sum of the two issuers' accumulators (issuer 1
+            // has none when the item has a single step)
             if (!(ok = mbar_wait(&bars->acc_full, item_it & 1, abort, p.status))) break;
             tc_fence_after();
             {
@@ -702,14 +713,18 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 __nv_bfloat16* out = (w == 0 ? p.dv : p.dk) + ((long long)b * p.S + (long long)j * 64) * p.Hkv * kD +
                                      (long long)h * kD + d;
                 const long long key_stride = (long long)p.Hkv * kD;
+                const bool two = N > 1;
 #pragma unroll 1
                 for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + 256 + 64 * w + 32 * hf, v);
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tmem + lane_base + 256 + 64 * w + 32 * hf, v0);
+                    tmem_ld32(tmem + lane_base + 384 + 64 * w + 32 * hf, v1);
                     tmem_wait_ld();
                     __nv_bfloat16* o2 = out + 32 * hf * key_stride;
 #pragma unroll 8
-                    for (int u = 0; u < 32; ++u) o2[u * key_stride] = __float2bfloat16_rn(__uint_as_float(v[u]));
+                    for (int u = 0; u < 32; ++u)
+                        o2[u * key_stride] =
+                            __float2bfloat16_rn(__uint_as_float(v0[u]) + (two ? __uint_as_float(v1[u]) : 0.f));
                 }
             }
             tc_fence_before();

@@ -10,10 +10,12 @@
 // query heads of a GQA group share the kept blocks, so one K/V block feeds
 // both Q tiles. Persistent grid; items in order of decreasing cost.
 //
-// One step = one kept block (64 keys). Warp roles (320 threads):
+// One step = one kept block (64 keys). Warp roles (352 threads):
 //   warp 0      TMA producer: the Q tiles once per item, then K and V of one
 //               block per step into a 4-stage ring (128B-swizzled).
-//   warp 1      TMEM owner and tcgen05 issuer (one thread): S_t = Q_t K^T
+//   warps 1, 10 tcgen05 issuers (one thread each), warp 1 for Q tile 0 (and
+//               TMEM owner), warp 10 for tile 1: a single thread issues MMAs
+//               at a bounded rate, so each tile has its own. S_t = Q_t K^T
 //               into one of two S buffers per tile, O_t += P_t V with P read
 //               from TMEM. S of step j+2 is issued as soon as PV of step j is,
 //               so the softmax of step j+1 never waits for an MMA.
@@ -34,7 +36,8 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kNS = 4;                              // K/V stages (one block each)
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
+constexpr int kIssuer1Warp = 10;                  // MMA issuer of Q tile 1
 constexpr uint32_t kBox = 64 * 128;                 // one TMA box: 64 rows x 128 B
 constexpr uint32_t kQAtom = 2 * kBox;               // 128 rows x 128 B
 constexpr uint32_t kQTile = 2 * kQAtom;             // 128 rows x 256 B
@@ -59,7 +62,7 @@ struct Bars {
     uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
     uint64_t s_full[2][2], p_full[2][2];
     uint64_t o_done[2], o_empty[2];
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -127,11 +130,11 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->q_empty, 2);                   // one arrival per MMA issuer
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
+            mbar_init(&bars->kv_empty[s], 2);
         }
         for (int t = 0; t < 2; ++t) {
             for (int b = 0; b < 2; ++b) {
@@ -141,7 +144,8 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mbar_init(&bars->o_done[t], 1);
             mbar_init(&bars->o_empty[t], 128);
         }
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -209,23 +213,36 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 if (q_issued) mbar_wait(&bars->q_full, (q_it - 1) & 1, &no_abort, nullptr);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == kIssuer1Warp) {
+        // ------------------------------------------------------------ MMA issuers, one per Q tile
+        // (one thread issues tcgen05.mma at a bounded rate, so each tile has its own)
         if (lane == 0) {
+            const int t = (warp == 1) ? 0 : 1;
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_pv = idesc_bf16(128, kD, false, true);
-            uint32_t kv_it = 0, q_it = 0, p_it[2][2] = {{0, 0}, {0, 0}}, oe_it[2] = {0, 0};
-            auto issue_s = [&](int t, int st, int buf) {
+            uint32_t kv_it = 0, q_it = 0, p_it[2] = {0, 0}, oe_it = 0;
+            constexpr uint32_t kHi = sdesc_hi(1024);
+            const uint32_t q_lo = sdesc_lo(sQ + t * kQTile, 16);
+            auto issue_s = [&](int st, int buf) {
+                const uint32_t k_lo = sdesc_lo(sKV + st * kStage, 16);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t a = sw128_desc(sQ + t * kQTile + (kk >> 2) * kQAtom + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = sw128_desc(sKV + st * kStage + (kk >> 2) * kBlkAtom + (kk & 3) * 32, 16, 1024);
-                    mma_ss(tmem + 256 * t + 64 * buf, a, b, id_s, kk > 0);
+                    const uint32_t ao = (kk >> 2) * kQAtom + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                    mma_ss_w(tmem + 256 * t + 64 * buf, q_lo + (ao >> 4), kHi, k_lo + (bo >> 4), kHi, id_s, kk > 0);
                 }
+                mma_commit(&bars->s_full[t][buf]);
             };
             bool ok = true;
             for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
                 const Item it = item_of(p, id);
+                if (t >= it.nt) {                       // tile 1 idle: tile 0's issuer arrives for it
+                    kv_it += it.nb;
+                    ++q_it;
+                    continue;
+                }
+                // arrivals this issuer owes the stage / Q barriers (2 when it is alone)
+                const int owe = (it.nt == 1) ? 2 : 1;
                 if (!(ok = mbar_wait(&bars->q_full, q_it & 1, abort, p.status))) break;
                 ++q_it;
                 tc_fence_after();
@@ -234,54 +251,45 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     const uint32_t g = kv_it + k;
                     if (!(ok = mbar_wait(&bars->k_full[g % kNS], (g / kNS) & 1, abort, p.status))) break;
                     tc_fence_after();
-                    for (int t = 0; t < it.nt; ++t) {
-                        issue_s(t, g % kNS, k & 1);
-                        mma_commit(&bars->s_full[t][k & 1]);
-                    }
+                    issue_s(g % kNS, k & 1);
                 }
                 if (!ok) break;
-                if (it.nb <= 2) mma_commit(&bars->q_empty);
+                if (it.nb <= 2)
+                    for (int c = 0; c < owe; ++c) mma_commit(&bars->q_empty);
                 for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
                     const int st = kv_it % kNS;
                     const int buf = k & 1;
                     if (!(ok = mbar_wait(&bars->v_full[st], (kv_it / kNS) & 1, abort, p.status))) break;
-                    tc_fence_after();
-                    const bool more = k + 2 < it.nb;
-                    const uint32_t g2 = kv_it + 2;
-                    for (int t = 0; t < it.nt && ok; ++t) {
-                        if (!(ok = mbar_wait(&bars->p_full[t][buf], p_it[t][buf] & 1, abort, p.status))) break;
-                        ++p_it[t][buf];
-                        if (k == 0) {
-                            if (!(ok = mbar_wait(&bars->o_empty[t], (oe_it[t] & 1) ^ 1, abort, p.status))) break;
-                            ++oe_it[t];
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + 256 * t + 128, tmem + 256 * t + 64 * buf + kk * 8,
-                                   sw128_desc(sKV + st * kStage + kBlk + kk * 2048, kBlkAtom, 1024), id_pv,
-                                   (k > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&bars->o_done[t]);
-                        if (more) {
-                            if (t == 0) {
-                                if (!(ok = mbar_wait(&bars->k_full[g2 % kNS], (g2 / kNS) & 1, abort, p.status)))
-                                    break;
-                                tc_fence_after();
-                            }
-                            issue_s(t, g2 % kNS, buf);
-                            mma_commit(&bars->s_full[t][buf]);
-                        }
+                    if (!(ok = mbar_wait(&bars->p_full[t][buf], p_it[buf] & 1, abort, p.status))) break;
+                    ++p_it[buf];
+                    if (k == 0) {
+                        if (!(ok = mbar_wait(&bars->o_empty[t], (oe_it & 1) ^ 1, abort, p.status))) break;
+                        ++oe_it;
                     }
-                    if (!ok) break;
-                    if (k + 3 == it.nb) mma_commit(&bars->q_empty);
-                    mma_commit(&bars->kv_empty[st]);
+                    tc_fence_after();
+                    const uint32_t v_lo = sdesc_lo(sKV + st * kStage + kBlk, kBlkAtom);   // MN-major V
+                    const uint32_t acc0 = k > 0 ? 1u : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts_w(tmem + 256 * t + 128, tmem + 256 * t + 64 * buf + kk * 8, v_lo + ((kk * 2048) >> 4),
+                                 kHi, id_pv, kk > 0 ? 1u : acc0);
+                    mma_commit(&bars->o_done[t]);
+                    if (k + 2 < it.nb) {
+                        const uint32_t g2 = kv_it + 2;
+                        if (!(ok = mbar_wait(&bars->k_full[g2 % kNS], (g2 / kNS) & 1, abort, p.status))) break;
+                        tc_fence_after();
+                        issue_s(g2 % kNS, buf);
+                    }
+                    if (k + 3 == it.nb)
+                        for (int c = 0; c < owe; ++c) mma_commit(&bars->q_empty);
+                    for (int c = 0; c < owe; ++c) mma_commit(&bars->kv_empty[st]);
                 }
             }
-            mma_commit(&bars->drain);
+            mma_commit(&bars->drain[t]);
             volatile int no_abort = 0;
-            mbar_wait(&bars->drain, 0, &no_abort, nullptr);
+            mbar_wait(&bars->drain[t], 0, &no_abort, nullptr);
         }
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         // ------------------------------------------------------------ softmax / epilogue
         const int t = (warp - 2) >> 2;                  // Q tile of this warpgroup
         const int quarter = warp & 3;                   // TMEM lane quarter this warp may access

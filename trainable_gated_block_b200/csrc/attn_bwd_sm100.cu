@@ -360,7 +360,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                             for (int q = 0; q < 2; ++q) {
                                 const int e = 8 * c + 2 * e2 + q;
                                 const bool live = row_ok && bk.valid && !(bk.cur && 32 * hf + e > r_in);
-                                const float pr = live ? exp2f(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
+                                const float pr = live ? fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
                                 const float ds = pr * (__uint_as_float(pv[e]) - drow);
                                 gs += ds;
                                 d2[q] = ds * p.sm_scale;
@@ -688,7 +688,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                             for (int q = 0; q < 2; ++q) {
                                 const int e = 8 * c + 2 * e2 + q;
                                 const bool live = sm.row_ok && !(sm.cur && 32 * hf + e > r_in);
-                                pr2[q] = live ? exp2f(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
+                                pr2[q] = live ? fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
                                 ds2[q] = pr2[q] * (__uint_as_float(pv[e]) - sm.drow) * p.sm_scale;
                             }
                             pp[e2] = pack_bf16x2(pr2[0], pr2[1]);

@@ -363,8 +363,8 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 uint32_t pk[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float p0 = exp2f(x[2 * e] - m_use);
-                    const float p1 = exp2f(x[2 * e + 1] - m_use);
+                    const float p0 = fast_exp2(x[2 * e] - m_use);
+                    const float p1 = fast_exp2(x[2 * e + 1] - m_use);
                     l += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }

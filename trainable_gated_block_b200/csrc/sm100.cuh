@@ -234,6 +234,15 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
     return (uint32_t)r * 128u + ((uint32_t)(c ^ (r & 7)) << 4);
 }
 
+// 2^x by the hardware approximation (one MUFU instruction; relative error
+// about 2^-22, subnormal results flushed to zero). Used for probabilities
+// that are rounded to bf16 or summed in fp32 right after.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

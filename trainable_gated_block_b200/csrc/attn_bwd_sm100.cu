@@ -35,10 +35,14 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-// warp 0 TMA, warps 1 and 10 MMA issuers (one thread each: a single thread
-// issues tcgen05.mma at a bounded rate), warps 2-5 / 6-9 two warpgroups
-constexpr int kThreads = 352;
-constexpr int kIssuer1Warp = 10;
+// warp 0 TMA, warps 2-5 / 6-9 two softmax warpgroups, warps 1, 10, 11, 12
+// four MMA-issuing warps (converged, elect.sync): one warp sustains about
+// one tcgen05.mma per ~125 cycles whatever the tile width, so the MMAs of a
+// step are spread over four warps that issue in parallel
+constexpr int kThreads = 416;
+__device__ __forceinline__ bool is_issuer_warp(int warp) { return warp == 1 || warp >= 10; }
+// issuer slot 0..3 of an issuing warp: warps 1, 10, 11, 12
+__device__ __forceinline__ int issuer_slot(int warp) { return warp == 1 ? 0 : warp - 9; }
 constexpr uint32_t kBox = 64 * 128;        // TMA box: 64 rows x 128 B
 constexpr uint32_t kTileAtom = 2 * kBox;   // 128 rows x 128 B (one 64-column half of a Q/dO tile)
 constexpr uint32_t kTile = 2 * kTileAtom;  // 128 rows x 256 B
@@ -89,7 +93,7 @@ struct Bars {
     uint64_t qd_full, qd_empty;
     uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
     uint64_t s_full[2], tm_free[2], ds_full[2], ds_empty[2], dq_full[2], dq_empty[2];
-    uint64_t drain[2];
+    uint64_t drain[4];
     uint32_t tmem_base;
     int abort;
 };
@@ -124,10 +128,11 @@ __device__ __forceinline__ Blk block_at(const Params& p, const Item& it, int k) 
     Blk r;
     if (k < it.c) {
         const int j = __ldg(p.idx + it.row * p.K + k);
+        const float lg = __ldg(p.log_gate + it.row * p.K + k);   // issued without waiting for j
         r.valid = (j >= 0 && j < it.i);
         r.j = r.valid ? j : it.i;
         r.cur = false;
-        r.bias2 = r.valid ? __ldg(p.log_gate + it.row * p.K + k) * kLog2e : 0.f;
+        r.bias2 = r.valid ? lg * kLog2e : 0.f;
     } else {
         r.j = it.i;
         r.valid = true;
@@ -147,21 +152,21 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
     volatile int* abort = &bars->abort;
     if (threadIdx.x == 0) {
         mbar_init(&bars->qd_full, 1);
-        mbar_init(&bars->qd_empty, 2);                  // one arrival per MMA issuer
+        mbar_init(&bars->qd_empty, 4);                  // one arrival per issuing warp
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 2);
+            mbar_init(&bars->kv_empty[s], 4);
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->s_full[t], 2);             // S and dP come from two warps
             mbar_init(&bars->tm_free[t], 128);
             mbar_init(&bars->ds_full[t], 128);
             mbar_init(&bars->ds_empty[t], 1);
             mbar_init(&bars->dq_full[t], 1);
             mbar_init(&bars->dq_empty[t], 128);
-            mbar_init(&bars->drain[t], 1);
         }
+        for (int w = 0; w < 4; ++w) mbar_init(&bars->drain[w], 1);
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -224,68 +229,65 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                 if (q_issued) mbar_wait(&bars->qd_full, (q_it - 1) & 1, &no_abort, nullptr);
             }
         }
-    } else if (warp == 1 || warp == kIssuer1Warp) {
-        if (lane == 0) {
-            const int t = (warp == 1) ? 0 : 1;          // the Q tile this thread issues for
-            const uint32_t id_s = idesc_bf16(128, 64, false, false);
-            const uint32_t id_dq = idesc_bf16(128, kD, false, true);
-            uint32_t kv_it = 0, q_it = 0, ds_it = 0, de_it = 0, sdp_n = 0;
-            bool ok = true;
-            const uint32_t q_lo = sdesc_lo(sQ + t * kTile, 16), o_lo = sdesc_lo(sO + t * kTile, 16);
-            // S and dP of this tile for the block in stage st, once its TMEM columns are free
-            auto issue_sdp = [&](int st) -> bool {
-                if (sdp_n > 0 && !mbar_wait(&bars->tm_free[t], (sdp_n - 1) & 1, abort, p.status)) return false;
-                ++sdp_n;
-                tc_fence_after();
-                const uint32_t kv_lo = sdesc_lo(sKV + st * kStage, 16);
+    } else if (is_issuer_warp(warp)) {
+        // slot 0 / 1: S and dQ of tile 0 / 1 (reads Q, K, dS); slot 2 / 3: dP of
+        // tile 0 / 1 (reads dO, V). The whole warp runs the loop, one lane issues.
+        const int slot = issuer_slot(warp);
+        const int t = slot & 1;                         // the Q tile this warp issues for
+        const bool sq = slot < 2;
+        const uint32_t id_s = idesc_bf16(128, 64, false, false);
+        const uint32_t id_dq = idesc_bf16(128, kD, false, true);
+        const uint32_t a_lo = sdesc_lo((sq ? sQ : sO) + t * kTile, 16);
+        const uint32_t d_sp = tmem + 256 * t + (sq ? 0u : 64u);
+        const uint32_t b_off = sq ? 0u : kBlk;          // K or V inside a stage
+        uint32_t kv_it = 0, q_it = 0, ds_it = 0, de_it = 0, sdp_n = 0;
+        bool ok = true;
+        // S (or dP) of this tile for the block in stage st, once the warpgroup has
+        // read the previous one out of TMEM
+        auto issue_sp = [&](int st) -> bool {
+            if (sdp_n > 0 && !mbar_wait_warp(&bars->tm_free[t], (sdp_n - 1) & 1, abort, p.status)) return false;
+            ++sdp_n;
+            tc_fence_after();
+            const uint32_t b_lo = sdesc_lo(sKV + st * kStage + b_off, 16);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                    mma_ss_w(tmem + 256 * t, q_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi, id_s, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                    const uint32_t bo = kBlk + (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                    mma_ss_w(tmem + 256 * t + 64, o_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi, id_s, kk > 0);
-                }
-                mma_commit(&bars->s_full[t]);
-                return true;
-            };
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
-                const Item it = item_of(p, id);
-                if (t >= it.nt) {                       // tile 1 idle: tile 0's issuer arrives for it
-                    kv_it += it.nb;
-                    ++q_it;
-                    continue;
-                }
-                const int owe = (it.nt == 1) ? 2 : 1;   // arrivals owed to the shared stage barriers
-                if (!(ok = mbar_wait(&bars->qd_full, q_it & 1, abort, p.status))) break;
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                mma_ss_e(d_sp, a_lo + (ao >> 4), kHi, b_lo + (bo >> 4), kHi, id_s, kk > 0);
+            }
+            mma_commit_e(&bars->s_full[t]);
+            return true;
+        };
+        auto wait_stage = [&](uint32_t n) -> bool {
+            const int st = n % kNS;
+            return mbar_wait_warp(sq ? &bars->k_full[st] : &bars->v_full[st], (n / kNS) & 1, abort, p.status);
+        };
+        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
+            const Item it = item_of(p, id);
+            if (t >= it.nt) {                       // tile 1 idle: tile 0's warps arrive for it
+                kv_it += it.nb;
                 ++q_it;
-                {
-                    const int st0 = kv_it % kNS;
-                    const uint32_t ph = (kv_it / kNS) & 1;
-                    if (!(ok = mbar_wait(&bars->k_full[st0], ph, abort, p.status))) break;
-                    if (!(ok = mbar_wait(&bars->v_full[st0], ph, abort, p.status))) break;
-                    if (!(ok = issue_sdp(st0))) break;
-                    if (it.nb == 1)
-                        for (int c = 0; c < owe; ++c) mma_commit(&bars->qd_empty);
+                continue;
+            }
+            const int owe = (it.nt == 1) ? 2 : 1;   // arrivals owed to the shared stage barriers
+            if (!(ok = mbar_wait_warp(&bars->qd_full, q_it & 1, abort, p.status))) break;
+            ++q_it;
+            if (!(ok = wait_stage(kv_it) && issue_sp(kv_it % kNS))) break;
+            if (it.nb == 1)
+                for (int c = 0; c < owe; ++c) mma_commit_e(&bars->qd_empty);
+            for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
+                const int st = kv_it % kNS;
+                const bool more = k + 1 < it.nb;
+                if (more) {                         // one block ahead
+                    if (!(ok = wait_stage(kv_it + 1) && issue_sp((kv_it + 1) % kNS))) break;
+                    if (k + 2 == it.nb)             // that was the last MMA reading this Q (dO) tile
+                        for (int c = 0; c < owe; ++c) mma_commit_e(&bars->qd_empty);
                 }
-                for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
-                    const int st = kv_it % kNS;
-                    const bool more = k + 1 < it.nb;
-                    if (more) {
-                        const int st1 = (kv_it + 1) % kNS;
-                        const uint32_t ph1 = ((kv_it + 1) / kNS) & 1;
-                        if (!(ok = mbar_wait(&bars->k_full[st1], ph1, abort, p.status))) break;
-                        if (!(ok = mbar_wait(&bars->v_full[st1], ph1, abort, p.status))) break;
-                        if (!(ok = issue_sdp(st1))) break;
-                    }
-                    if (!(ok = mbar_wait(&bars->ds_full[t], ds_it & 1, abort, p.status))) break;
+                if (sq) {
+                    if (!(ok = mbar_wait_warp(&bars->ds_full[t], ds_it & 1, abort, p.status))) break;
                     ++ds_it;
                     if (k == 0) {
-                        if (!(ok = mbar_wait(&bars->dq_empty[t], (de_it & 1) ^ 1, abort, p.status))) break;
+                        if (!(ok = mbar_wait_warp(&bars->dq_empty[t], (de_it & 1) ^ 1, abort, p.status))) break;
                         ++de_it;
                     }
                     tc_fence_after();
@@ -294,19 +296,17 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     const uint32_t acc0 = k > 0 ? 1u : 0u;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ss_w(tmem + 256 * t + 128, ds_lo + ((kk * 32) >> 4), kHi, kt_lo + ((kk * 2048) >> 4), kHi,
+                        mma_ss_e(tmem + 256 * t + 128, ds_lo + ((kk * 32) >> 4), kHi, kt_lo + ((kk * 2048) >> 4), kHi,
                                  id_dq, kk > 0 ? 1u : acc0);
-                    mma_commit(&bars->ds_empty[t]);
-                    if (!more) mma_commit(&bars->dq_full[t]);
-                    if (k + 2 == it.nb)
-                        for (int c = 0; c < owe; ++c) mma_commit(&bars->qd_empty);
-                    for (int c = 0; c < owe; ++c) mma_commit(&bars->kv_empty[st]);
+                    mma_commit_e(&bars->ds_empty[t]);
+                    if (!more) mma_commit_e(&bars->dq_full[t]);
                 }
+                for (int c = 0; c < owe; ++c) mma_commit_e(&bars->kv_empty[st]);
             }
-            mma_commit(&bars->drain[t]);
-            volatile int no_abort = 0;
-            mbar_wait(&bars->drain[t], 0, &no_abort, nullptr);
         }
+        mma_commit_e(&bars->drain[slot]);
+        volatile int no_abort = 0;
+        mbar_wait(&bars->drain[slot], 0, &no_abort, nullptr);
     } else if (warp >= 2 && warp < 10) {
         const int t = (warp - 2) >> 2;
         const int quarter = warp & 3;
@@ -335,7 +335,9 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                 if (!(ok = mbar_wait(&bars->s_full[t], s_it & 1, abort, p.status))) break;
                 ++s_it;
                 tc_fence_after();
-                const float off = bk.bias2 - lse2;
+                // log2 domain; rows of an absent head (or a bad block) get -inf: P = dS = 0
+                const float off = (row_ok && bk.valid) ? bk.bias2 - lse2 : -INFINITY;
+                const int lim = bk.cur ? r_in : 63;       // causal mask on the diagonal block
                 float gs = 0.f;
                 // dQ of the previous step has finished reading the dS tile
                 if (ds_n > 0 && !(ok = mbar_wait(&bars->ds_empty[t], (ds_n - 1) & 1, abort, p.status))) break;
@@ -359,8 +361,9 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
 #pragma unroll
                             for (int q = 0; q < 2; ++q) {
                                 const int e = 8 * c + 2 * e2 + q;
-                                const bool live = row_ok && bk.valid && !(bk.cur && 32 * hf + e > r_in);
-                                const float pr = live ? fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
+                                float x = fmaf(__uint_as_float(sv[e]), p.scale2, off);
+                                x = (32 * hf + e > lim) ? -INFINITY : x;
+                                const float pr = fast_exp2(x);
                                 const float ds = pr * (__uint_as_float(pv[e]) - drow);
                                 gs += ds;
                                 d2[q] = ds * p.sm_scale;
@@ -432,7 +435,7 @@ struct Bars {
     uint64_t qd_full[kNS], qd_empty[kNS];
     uint64_t s_full[2], tm_free[2], pds_full[2], pds_empty[2];
     uint64_t acc_full, acc_empty;
-    uint64_t drain[2];
+    uint64_t drain[4];
     uint32_t tmem_base;
     int abort;
 };
@@ -452,33 +455,31 @@ __device__ __forceinline__ int n_entries(const Params& p, long long bh, int j) {
 
 // What a softmax thread needs for step m of item (b, h, j): the query block,
 // the gate of block j in that block's selection, and its row's LSE and Dr.
+// The reverse-list entry of a step is loaded two steps ahead and the loads
+// that depend on it one step ahead, all independent of each other (no load
+// address waits on another load's value inside a step).
 struct StepMeta {
-    int i;
-    bool cur, row_ok;
-    float bias2, lse2, drow;
+    bool cur, in_range, row_ok;
+    int slot, idxv;
+    float lg, lse, drow;
 };
-__device__ __forceinline__ StepMeta step_meta(const Params& p, const int32_t* list, int b, int h, long long bh, int j,
-                                              int m, int row) {
+__device__ __forceinline__ StepMeta step_meta(const Params& p, int ent, int b, int h, long long bh, int j, int m,
+                                              int row) {
     StepMeta s;
-    const int e = m / p.ntile, t = m % p.ntile;
-    const int ent = __ldg(list + e);
+    const int t = m % p.ntile;
     int i = ent >> 16;
-    const int slot = ent & 0xFFFF;
-    bool valid = i >= j && i < p.NQB;
-    if (!valid) i = j;
-    s.i = i;
+    s.slot = ent & 0xFFFF;
+    s.in_range = i >= j && i < p.NQB;
+    if (!s.in_range) i = j;
     s.cur = (i == j);
-    s.bias2 = 0.f;
-    if (!s.cur) {
-        const long long srow = bh * p.NQB + i;
-        valid = valid && slot < p.K && __ldg(p.idx + srow * p.K + slot) == j;
-        s.bias2 = valid ? __ldg(p.log_gate + srow * p.K + slot) * kLog2e : 0.f;
-    }
+    const long long sidx = (bh * p.NQB + i) * p.K + min(s.slot, p.K - 1);
+    s.idxv = s.cur ? j : __ldg(p.idx + sidx);
+    s.lg = s.cur ? 0.f : __ldg(p.log_gate + sidx);
     const int hs = 2 * t + (row >> 6);
-    s.row_ok = valid && hs < p.G;
-    const int hq = h * p.G + (hs < p.G ? hs : 0);
+    s.row_ok = hs < p.G;
+    const int hq = h * p.G + (s.row_ok ? hs : 0);
     const long long lrow = ((long long)b * p.Hq + hq) * p.S + (long long)i * 64 + (row & 63);
-    s.lse2 = __ldg(p.lse + lrow) * kLog2e;
+    s.lse = __ldg(p.lse + lrow);
     s.drow = __ldg(p.Dr + lrow);
     return s;
 }
@@ -493,19 +494,19 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     volatile int* abort = &bars->abort;
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
-        mbar_init(&bars->kv_empty, 2);                  // one arrival per MMA issuer
+        mbar_init(&bars->kv_empty, 4);                  // one arrival per issuing warp
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&bars->qd_full[s], 1);
-            mbar_init(&bars->qd_empty[s], 1);
+            mbar_init(&bars->qd_empty[s], 2);           // the two warps of the step's warpgroup
         }
         for (int w = 0; w < 2; ++w) {
-            mbar_init(&bars->s_full[w], 1);
+            mbar_init(&bars->s_full[w], 2);
             mbar_init(&bars->tm_free[w], 128);
             mbar_init(&bars->pds_full[w], 128);
-            mbar_init(&bars->pds_empty[w], 1);
-            mbar_init(&bars->drain[w], 1);
+            mbar_init(&bars->pds_empty[w], 2);
         }
-        mbar_init(&bars->acc_full, 2);
+        for (int w = 0; w < 4; ++w) mbar_init(&bars->drain[w], 1);
+        mbar_init(&bars->acc_full, 4);
         mbar_init(&bars->acc_empty, 256);
         bars->abort = 0;
         fence_barrier_init();
@@ -570,75 +571,71 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (kv_issued) mbar_wait(&bars->kv_full, (item_it - 1) & 1, &no_abort, nullptr);
             }
         }
-    } else if (warp == 1 || warp == kIssuer1Warp) {
-        // one issuer per warpgroup: issuer w runs the steps m = w, w+2, ... of each
-        // item and accumulates its own dV^T, dK^T (the drain adds the two)
-        if (lane == 0) {
-            const int w = (warp == 1) ? 0 : 1;
-            const uint32_t id_s = idesc_bf16(128, 64, false, false);
-            const uint32_t id_t = idesc_bf16(128, 64, true, true);
-            const uint32_t k_lo = sdesc_lo(s_base + kOffK, 16), v_lo = sdesc_lo(s_base + kOffV, 16);
-            const uint32_t plo = sdesc_lo(s_base + kOffPS + w * 2 * kRowTile, kRowTile);   // P, dS (MN-major)
-            const uint32_t acc_v = tmem + 256 + 128 * w, acc_k = acc_v + 64;
-            uint32_t item_it = 0, gbase = 0, pds_it = 0, sdp_n = 0;
-            bool ok = true;
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
-                int b, h, j;
-                long long bh;
-                item_of(p, id, b, h, j, bh);
-                const int N = n_entries(p, bh, j) * p.ntile;
-                if (!(ok = mbar_wait(&bars->kv_full, item_it & 1, abort, p.status))) break;
-                // the drain of the previous item has read both accumulators
-                if (!(ok = mbar_wait(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
+    } else if (is_issuer_warp(warp)) {
+        // Step m of an item belongs to warpgroup w = m % 2. For warpgroup w, slot w
+        // issues S = Q K^T and dK^T += Q^T dS, slot 2 + w issues dP = dO V^T and
+        // dV^T += dO^T P, each into its own accumulator (the drain adds the two
+        // warpgroups' halves). The whole warp runs the loop, one lane issues.
+        const int slot = issuer_slot(warp);
+        const int w = slot & 1;
+        const bool xq = slot < 2;                       // the Q side (else the dO side)
+        const uint32_t id_s = idesc_bf16(128, 64, false, false);
+        const uint32_t id_t = idesc_bf16(128, 64, true, true);
+        const uint32_t kv_lo = sdesc_lo(s_base + (xq ? kOffK : kOffV), 16);
+        const uint32_t a_off = xq ? 0u : kTile;         // Q or dO inside a stage
+        const uint32_t d_sp = tmem + 128 * w + (xq ? 0u : 64u);
+        // accumulator: dV^T of warpgroup w at 256 + 128 w, dK^T at + 64
+        const uint32_t acc = tmem + 256 + 128 * w + (xq ? 64u : 0u);
+        // B of the accumulation: P (dO side) or dS (Q side) of warpgroup w, MN-major
+        const uint32_t pb_lo = sdesc_lo(s_base + kOffPS + w * 2 * kRowTile + (xq ? kRowTile : 0u), kRowTile);
+        uint32_t item_it = 0, gbase = 0, pds_it = 0, sdp_n = 0;
+        bool ok = true;
+        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+            int b, h, j;
+            long long bh;
+            item_of(p, id, b, h, j, bh);
+            const int N = n_entries(p, bh, j) * p.ntile;
+            if (!(ok = mbar_wait_warp(&bars->kv_full, item_it & 1, abort, p.status))) break;
+            // the drain of the previous item has read both accumulators
+            if (!(ok = mbar_wait_warp(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
+            tc_fence_after();
+            for (int m = w; m < N && ok; m += 2) {
+                const uint32_t g = gbase + m;
+                const int st = g % kNS;
+                if (!(ok = mbar_wait_warp(&bars->qd_full[st], (g / kNS) & 1, abort, p.status))) break;
+                // this warpgroup has loaded its previous S/dP out of TMEM
+                if (sdp_n > 0 && !(ok = mbar_wait_warp(&bars->tm_free[w], (sdp_n - 1) & 1, abort, p.status))) break;
+                ++sdp_n;
                 tc_fence_after();
-                for (int m = w; m < N && ok; m += 2) {
-                    const uint32_t g = gbase + m;
-                    const int st = g % kNS;
-                    if (!(ok = mbar_wait(&bars->qd_full[st], (g / kNS) & 1, abort, p.status))) break;
-                    // this warpgroup has loaded its previous S/dP out of TMEM
-                    if (sdp_n > 0 && !(ok = mbar_wait(&bars->tm_free[w], (sdp_n - 1) & 1, abort, p.status))) break;
-                    ++sdp_n;
-                    tc_fence_after();
-                    const uint32_t qk = sdesc_lo(s_base + kOffStage + st * kStage, 16);   // K-major Q, dO
+                const uint32_t a_lo = sdesc_lo(s_base + kOffStage + st * kStage + a_off, 16);   // K-major Q / dO
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                        const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                        mma_ss_w(tmem + 128 * w, qk + (ao >> 4), kHi, k_lo + (bo >> 4), kHi, id_s, kk > 0);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ao = kTile + (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                        const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                        mma_ss_w(tmem + 128 * w + 64, qk + (ao >> 4), kHi, v_lo + (bo >> 4), kHi, id_s, kk > 0);
-                    }
-                    mma_commit(&bars->s_full[w]);
-                    // dV^T += dO^T P, dK^T += Q^T dS once the warpgroup wrote P and dS
-                    if (!(ok = mbar_wait(&bars->pds_full[w], pds_it & 1, abort, p.status))) break;
-                    ++pds_it;
-                    tc_fence_after();
-                    const uint32_t qlo = sdesc_lo(s_base + kOffStage + st * kStage, kTileAtom);   // MN-major Q, dO
-                    const uint32_t acc0 = (m >= 2) ? 1u : 0u;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss_w(acc_v, qlo + ((kTile + kk * 2048) >> 4), kHi, plo + ((kk * 2048) >> 4), kHi, id_t,
-                                 kk > 0 ? 1u : acc0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss_w(acc_k, qlo + ((kk * 2048) >> 4), kHi, plo + ((kRowTile + kk * 2048) >> 4), kHi, id_t,
-                                 kk > 0 ? 1u : acc0);
-                    mma_commit(&bars->qd_empty[st]);
-                    mma_commit(&bars->pds_empty[w]);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                    mma_ss_e(d_sp, a_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi, id_s, kk > 0);
                 }
-                if (!ok) break;
-                gbase += N;
-                mma_commit(&bars->kv_empty);
-                mma_commit(&bars->acc_full);
+                mma_commit_e(&bars->s_full[w]);
+                // the accumulation once the warpgroup wrote P and dS
+                if (!(ok = mbar_wait_warp(&bars->pds_full[w], pds_it & 1, abort, p.status))) break;
+                ++pds_it;
+                tc_fence_after();
+                const uint32_t at_lo = sdesc_lo(s_base + kOffStage + st * kStage + a_off, kTileAtom);   // MN-major
+                const uint32_t acc0 = (m >= 2) ? 1u : 0u;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss_e(acc, at_lo + ((kk * 2048) >> 4), kHi, pb_lo + ((kk * 2048) >> 4), kHi, id_t,
+                             kk > 0 ? 1u : acc0);
+                mma_commit_e(&bars->qd_empty[st]);
+                mma_commit_e(&bars->pds_empty[w]);
             }
-            mma_commit(&bars->drain[w]);
-            volatile int no_abort = 0;
-            mbar_wait(&bars->drain[w], 0, &no_abort, nullptr);
+            if (!ok) break;
+            gbase += N;
+            mma_commit_e(&bars->kv_empty);
+            mma_commit_e(&bars->acc_full);
         }
+        mma_commit_e(&bars->drain[slot]);
+        volatile int no_abort = 0;
+        mbar_wait(&bars->drain[slot], 0, &no_abort, nullptr);
     } else if (warp >= 2 && warp < 10) {
         const int w = (warp - 2) >> 2;
         const int quarter = warp & 3;
@@ -656,30 +653,36 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             item_of(p, id, b, h, j, bh);
             const int N = n_entries(p, bh, j) * p.ntile;
             const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
+            // metadata pipeline: entry of step m + 4 and loads of step m + 2 in flight
+            int ent2 = (w + 2 < N) ? __ldg(list + (w + 2) / p.ntile) : 0;
             StepMeta nxt;
-            if (w < N) nxt = step_meta(p, list, b, h, bh, j, w, row);
+            if (w < N) nxt = step_meta(p, __ldg(list + w / p.ntile), b, h, bh, j, w, row);
             for (int m = w; m < N; m += 2) {
                 const StepMeta sm = nxt;
-                if (m + 2 < N) nxt = step_meta(p, list, b, h, bh, j, m + 2, row);   // prefetch
+                if (m + 2 < N) nxt = step_meta(p, ent2, b, h, bh, j, m + 2, row);
+                if (m + 4 < N) ent2 = __ldg(list + (m + 4) / p.ntile);
                 if (!(ok = mbar_wait(&bars->s_full[w], s_it & 1, abort, p.status))) break;
                 ++s_it;
                 tc_fence_after();
-                const float off = sm.bias2 - sm.lse2;
+                const bool valid = sm.in_range && (sm.cur || (sm.slot < p.K && sm.idxv == j));
+                // log2 domain; rows of an absent head (or a bad entry) get -inf: P = dS = 0
+                const float off = (valid && sm.row_ok) ? sm.lg * kLog2e - sm.lse * kLog2e : -INFINITY;
+                const int lim = sm.cur ? r_in : 63;       // causal mask on the diagonal block
                 // the MMA of this warpgroup's previous step has finished reading the buffers
                 if (pds_n > 0 && !(ok = mbar_wait(&bars->pds_empty[w], (pds_n - 1) & 1, abort, p.status))) break;
                 ++pds_n;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {          // keys [32 hf, 32 hf + 32)
-                    uint32_t sv[32], pv[32];
-                    tmem_ld32(tS + 32 * hf, sv);
-                    tmem_ld32(tS + 64 + 32 * hf, pv);
+                for (int qt = 0; qt < 4; ++qt) {          // keys [16 qt, 16 qt + 16)
+                    uint32_t sv[16], pv[16];
+                    tmem_ld16(tS + 16 * qt, sv);
+                    tmem_ld16(tS + 64 + 16 * qt, pv);
                     tmem_wait_ld();
-                    if (hf == 1) {
+                    if (qt == 3) {
                         tc_fence_before();
                         mbar_arrive(&bars->tm_free[w]);   // S/dP columns may be refilled
                     }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {         // 16-byte chunk = keys 8c .. 8c+7 of the half
+                    for (int c = 0; c < 2; ++c) {         // 16-byte chunk = keys 8c .. 8c+7 of the quarter
                         uint32_t pp[4], dd[4];
 #pragma unroll
                         for (int e2 = 0; e2 < 4; ++e2) {
@@ -687,14 +690,15 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 #pragma unroll
                             for (int q = 0; q < 2; ++q) {
                                 const int e = 8 * c + 2 * e2 + q;
-                                const bool live = sm.row_ok && !(sm.cur && 32 * hf + e > r_in);
-                                pr2[q] = live ? fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale2, off)) : 0.f;
-                                ds2[q] = pr2[q] * (__uint_as_float(pv[e]) - sm.drow) * p.sm_scale;
+                                float x = fmaf(__uint_as_float(sv[e]), p.scale2, off);
+                                x = (16 * qt + e > lim) ? -INFINITY : x;
+                                pr2[q] = fast_exp2(x);
+                                ds2[q] = (pr2[q] * p.sm_scale) * (__uint_as_float(pv[e]) - sm.drow);
                             }
                             pp[e2] = pack_bf16x2(pr2[0], pr2[1]);
                             dd[e2] = pack_bf16x2(ds2[0], ds2[1]);
                         }
-                        const int ch = 4 * hf + c;
+                        const int ch = 2 * qt + c;
                         *reinterpret_cast<uint4*>(bufP + sw128_offset(row, ch)) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
                         *reinterpret_cast<uint4*>(bufS + sw128_offset(row, ch)) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
                     }
@@ -715,14 +719,14 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 const long long key_stride = (long long)p.Hkv * kD;
                 const bool two = N > 1;
 #pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(tmem + lane_base + 256 + 64 * w + 32 * hf, v0);
-                    tmem_ld32(tmem + lane_base + 384 + 64 * w + 32 * hf, v1);
+                for (int qt = 0; qt < 4; ++qt) {
+                    uint32_t v0[16], v1[16];
+                    tmem_ld16(tmem + lane_base + 256 + 64 * w + 16 * qt, v0);
+                    tmem_ld16(tmem + lane_base + 384 + 64 * w + 16 * qt, v1);
                     tmem_wait_ld();
-                    __nv_bfloat16* o2 = out + 32 * hf * key_stride;
-#pragma unroll 8
-                    for (int u = 0; u < 32; ++u)
+                    __nv_bfloat16* o2 = out + 16 * qt * key_stride;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
                         o2[u * key_stride] =
                             __float2bfloat16_rn(__uint_as_float(v0[u]) + (two ? __uint_as_float(v1[u]) : 0.f));
                 }

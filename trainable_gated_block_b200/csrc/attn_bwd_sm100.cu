@@ -63,6 +63,7 @@ struct Params {
     const int32_t* rcount;  // [B, Hkv, NQB]
     float scale2;           // sm_scale * log2(e)
     float sm_scale;
+    float inv_scale;        // 1 / sm_scale
     __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -70,11 +71,41 @@ struct Params {
     int* status;
 };
 
-// Writes 64 bf16 pairs-packed values (one 128-byte row) into a 128B-swizzled tile.
-__device__ __forceinline__ void store_row(uint8_t* tile, int row, const uint32_t (&v)[32]) {
+// Elementwise part of the backward for the 32 keys [32 hf, 32 hf + 32) of
+// one query row, from its S (sv) and dP (pv) values read out of TMEM:
+//   P = 2^(S * sm_scale * log2 e + off),  dS' = P * (dP * sm_scale - Dr * sm_scale)
+// where off = log2 g - lse (log2 units) or -inf for a dead row; keys above
+// `lim` are masked (the diagonal block, kMask). dS' (dS times sm_scale) is
+// rounded to bf16 into the row's 128-byte-swizzled tile, and P too when a P
+// tile is given. Returns the row's sum of dS'.
+template <bool kMask>
+__device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32_t (&pv)[32], int hf, float scale2,
+                                          float off, float sm_scale, float drs, int lim, uint8_t* bufP,
+                                          uint8_t* bufS, int row) {
+    float gs = 0.f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(tile + sw128_offset(row, c)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    for (int c = 0; c < 4; ++c) {                 // 16-byte chunk = keys 8c .. 8c+7 of the half
+        uint32_t pp[4], dd[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            float pr[2], ds[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int e = 8 * c + 2 * e2 + q;
+                float x = fmaf(__uint_as_float(sv[e]), scale2, off);
+                if (kMask) x = (32 * hf + e > lim) ? -INFINITY : x;
+                pr[q] = fast_exp2(x);
+                ds[q] = pr[q] * fmaf(__uint_as_float(pv[e]), sm_scale, -drs);
+                gs += ds[q];
+            }
+            pp[e2] = pack_bf16x2(pr[0], pr[1]);
+            dd[e2] = pack_bf16x2(ds[0], ds[1]);
+        }
+        const int ch = 4 * hf + c;
+        if (bufP) *reinterpret_cast<uint4*>(bufP + sw128_offset(row, ch)) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
+        *reinterpret_cast<uint4*>(bufS + sw128_offset(row, ch)) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
+    }
+    return gs;
 }
 
 // ===================================================================== dq
@@ -326,7 +357,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             const int hq = it.h * p.G + (row_ok ? slot : 0);
             const long long lrow = ((long long)it.b * p.Hq + hq) * p.S + (long long)it.i * 64 + r_in;
             const float lse2 = p.lse[lrow] * kLog2e;
-            const float drow = p.Dr[lrow];
+            const float drs = p.Dr[lrow] * p.sm_scale;
             bool ok = true;
             Blk nxt = block_at(p, it, 0);
             for (int k = 0; k < it.nb; ++k) {
@@ -337,8 +368,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                 tc_fence_after();
                 // log2 domain; rows of an absent head (or a bad block) get -inf: P = dS = 0
                 const float off = (row_ok && bk.valid) ? bk.bias2 - lse2 : -INFINITY;
-                const int lim = bk.cur ? r_in : 63;       // causal mask on the diagonal block
-                float gs = 0.f;
+                float gs = 0.f;                           // sum of dS * sm_scale over the row's keys
                 // dQ of the previous step has finished reading the dS tile
                 if (ds_n > 0 && !(ok = mbar_wait(&bars->ds_empty[t], (ds_n - 1) & 1, abort, p.status))) break;
                 ++ds_n;
@@ -352,33 +382,16 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                         tc_fence_before();
                         mbar_arrive(&bars->tm_free[t]);   // S/dP columns may be refilled
                     }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {         // 16-byte chunk = keys 8c .. 8c+7 of the half
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            float d2[2];
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const int e = 8 * c + 2 * e2 + q;
-                                float x = fmaf(__uint_as_float(sv[e]), p.scale2, off);
-                                x = (32 * hf + e > lim) ? -INFINITY : x;
-                                const float pr = fast_exp2(x);
-                                const float ds = pr * (__uint_as_float(pv[e]) - drow);
-                                gs += ds;
-                                d2[q] = ds * p.sm_scale;
-                            }
-                            pk[e2] = pack_bf16x2(d2[0], d2[1]);
-                        }
-                        *reinterpret_cast<uint4*>(ds_tile + sw128_offset(row, 4 * hf + c)) =
-                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
+                    if (bk.cur)                           // causal mask on the diagonal block
+                        gs += pds_half<true>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, r_in, nullptr, ds_tile, row);
+                    else
+                        gs += pds_half<false>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, 63, nullptr, ds_tile, row);
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&bars->ds_full[t]);
                 if (!bk.cur && bk.valid) {
                     gs = warp_sum(gs);
-                    if (lane == 0) atomicAdd(p.gsum + it.row * p.K + k, gs);
+                    if (lane == 0) atomicAdd(p.gsum + it.row * p.K + k, gs * p.inv_scale);
                 }
             }
             if (!ok) break;
@@ -667,41 +680,24 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 const bool valid = sm.in_range && (sm.cur || (sm.slot < p.K && sm.idxv == j));
                 // log2 domain; rows of an absent head (or a bad entry) get -inf: P = dS = 0
                 const float off = (valid && sm.row_ok) ? sm.lg * kLog2e - sm.lse * kLog2e : -INFINITY;
-                const int lim = sm.cur ? r_in : 63;       // causal mask on the diagonal block
+                const float drs = sm.drow * p.sm_scale;
                 // the MMA of this warpgroup's previous step has finished reading the buffers
                 if (pds_n > 0 && !(ok = mbar_wait(&bars->pds_empty[w], (pds_n - 1) & 1, abort, p.status))) break;
                 ++pds_n;
 #pragma unroll
-                for (int qt = 0; qt < 4; ++qt) {          // keys [16 qt, 16 qt + 16)
-                    uint32_t sv[16], pv[16];
-                    tmem_ld16(tS + 16 * qt, sv);
-                    tmem_ld16(tS + 64 + 16 * qt, pv);
+                for (int hf = 0; hf < 2; ++hf) {          // keys [32 hf, 32 hf + 32)
+                    uint32_t sv[32], pv[32];
+                    tmem_ld32(tS + 32 * hf, sv);
+                    tmem_ld32(tS + 64 + 32 * hf, pv);
                     tmem_wait_ld();
-                    if (qt == 3) {
+                    if (hf == 1) {
                         tc_fence_before();
                         mbar_arrive(&bars->tm_free[w]);   // S/dP columns may be refilled
                     }
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {         // 16-byte chunk = keys 8c .. 8c+7 of the quarter
-                        uint32_t pp[4], dd[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            float pr2[2], ds2[2];
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const int e = 8 * c + 2 * e2 + q;
-                                float x = fmaf(__uint_as_float(sv[e]), p.scale2, off);
-                                x = (16 * qt + e > lim) ? -INFINITY : x;
-                                pr2[q] = fast_exp2(x);
-                                ds2[q] = (pr2[q] * p.sm_scale) * (__uint_as_float(pv[e]) - sm.drow);
-                            }
-                            pp[e2] = pack_bf16x2(pr2[0], pr2[1]);
-                            dd[e2] = pack_bf16x2(ds2[0], ds2[1]);
-                        }
-                        const int ch = 2 * qt + c;
-                        *reinterpret_cast<uint4*>(bufP + sw128_offset(row, ch)) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
-                        *reinterpret_cast<uint4*>(bufS + sw128_offset(row, ch)) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
-                    }
+                    if (sm.cur)                           // causal mask on the diagonal block
+                        pds_half<true>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, r_in, bufP, bufS, row);
+                    else
+                        pds_half<false>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, 63, bufP, bufS, row);
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&bars->pds_full[w]);
@@ -875,6 +871,7 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     p.rcount = ws.rcount;
     p.scale2 = a.sm_scale * kLog2e;
     p.sm_scale = a.sm_scale;
+    p.inv_scale = 1.f / a.sm_scale;
     p.dq = static_cast<__nv_bfloat16*>(bw.dq);
     p.dk = static_cast<__nv_bfloat16*>(bw.dk);
     p.dv = static_cast<__nv_bfloat16*>(bw.dv);

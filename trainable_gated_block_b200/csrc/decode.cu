@@ -6,226 +6,467 @@
 // 64-token pages. Only the kept pages are read: each (page, KV head) is one
 // contiguous 16 KiB tile of K and one of V.
 //
-// Split-KV: CTA (split, h, n) walks up to kBps of the (cnt + 1) blocks of
-// (n, h) for all G query heads of the group, keeping an online softmax per
-// head in the log2 domain, and writes an unnormalised partial (m, l, o).
-// A combine kernel merges the splits. HBM-bound: every K/V byte is read once
-// with 16-byte non-coherent loads; the math is fp32 FMA on the CUDA cores.
+// HBM-bound design. Work item = (sequence n, KV head h) with its cnt + 1
+// blocks; the items' blocks are laid end to end ((K + 1) slots per item) and
+// cut into one contiguous range per CTA, so every SM streams the same number
+// of blocks. One persistent CTA per SM:
+//  * a producer warp resolves 32 slots at a time (selection entry -> page ->
+//    gate, in parallel over its lanes) and TMA-copies each kept (page, head)
+//    K and V tile, 128-byte swizzled, into a ring of six 32 KiB stages;
+//  * three consumer warps take the CTA's blocks round robin (warp w owns
+//    stages w and w + 3, so each warp's stages are double buffered). A warp
+//    does a whole block on the tensor cores with mma.sync m16n8k16: the G
+//    query heads of the group are the rows of the 16-row A operand (the
+//    rest zero), S = Q K^T over 64 keys (8 n-tiles x 8 k-steps), then an
+//    online softmax in the log2 domain on the S fragments (a row lives in
+//    the 4 lanes of a quad), then O += P V (16 n-tiles x 4 k-steps) with P
+//    taken straight from the S fragments. K and V fragments come from shared
+//    memory by ldmatrix (conflict-free on the swizzled layout);
+//  * when the CTA leaves an item, the warps' states are merged through
+//    shared memory into one partial (m, l, o) for that (item, CTA).
+// A combine kernel merges the (at most a few) partials of each query head.
+// The tensor work is tiny (the kernel is bound by HBM); using it keeps the
+// per-block instruction count low enough that the math hides under the
+// page reads.
 #include "common.cuh"
 #include "launch.h"
+#include "sm100.cuh"
 
 namespace sas {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kBps = 4;                 // blocks per split
+using namespace sm100;
+
 constexpr int kD = 128;
-constexpr int kKStride = kD + 8;        // bf16 elements per padded K row (272 B)
+constexpr int kWarps = 3;                          // consumer warps
+constexpr int kThreads = (kWarps + 1) * 32;        // + one producer warp
+constexpr int kStages = 2 * kWarps;                // warp w owns stages w and w + kWarps
+constexpr uint32_t kBoxBytes = 64 * 128;           // TMA box: 64 rows x 64 dims (128 B)
+constexpr uint32_t kTileBytes = 2 * kBoxBytes;     // one (page, head) tile of K or V
+constexpr uint32_t kStageBytes = 2 * kTileBytes;
+constexpr uint32_t kOffMo = kStages * kStageBytes;                 // merge scratch: o [warp][8][D]
+constexpr uint32_t kOffMl = kOffMo + kWarps * 8 * kD * 4;          // merge scratch: m, l [warp][8][2]
+constexpr uint32_t kOffMeta = kOffMl + kWarps * 8 * 2 * 4;         // per-stage (bias, valid keys)
+constexpr uint32_t kOffBar = kOffMeta + kStages * 8;
+constexpr uint32_t kSmem = kOffBar + 2 * kStages * 8 + 16 + 1024;  // + alignment slack
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 
-inline int num_splits(int K) { return (K + 1 + kBps - 1) / kBps; }
-
-struct Part {
-    float* o;       // [N, Hq, splits, D]
-    float* ml;      // [N, Hq, splits, 2]  (max, sum), log2 domain
+struct Params {
+    const __nv_bfloat16* q;
+    int num_pages;
+    const int32_t* page_table;
+    int max_pages;
+    const int32_t* kv_len;
+    int Hq, Hkv, G, K;
+    const int32_t* idx;
+    const int32_t* cnt;
+    const float* log_gate;
+    float qscale;           // sm_scale * log2(e)
+    long long V;            // n_items * (K + 1) block slots
+    int grid;
+    int nslot;              // partial slots per query head
+    float* part_o;          // [N * Hq, nslot, D]
+    float* part_ml;         // [N * Hq, nslot, 2]
+    int* status;
 };
 
-inline Part carve(void* ws, int N, int Hq, int K) {
-    Part p;
-    const size_t no = (size_t)N * Hq * num_splits(K) * kD;
-    p.o = static_cast<float*>(ws);
-    p.ml = p.o + no;
-    return p;
+// CTA c owns block slots [c V / grid, (c + 1) V / grid); cta_of is its inverse.
+__host__ __device__ __forceinline__ long long slot_begin(long long c, long long V, int grid) { return c * V / grid; }
+__host__ __device__ __forceinline__ int cta_of(long long s, long long V, int grid) {
+    return (int)(((s + 1) * grid - 1) / V);
 }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads)
-decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
-                    const __nv_bfloat16* __restrict__ vc, int num_pages,
-                    const int32_t* __restrict__ page_table, int max_pages,
-                    const int32_t* __restrict__ kv_len, int Hq, int Hkv, int K,
-                    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
-                    const float* __restrict__ log_gate, float sm_scale, Part part, int* status) {
-    constexpr int ITEMS = (G * 64 + kThreads - 1) / kThreads;   // (head, dim-pair) items per thread
-    __shared__ __align__(16) __nv_bfloat16 Ks[kBlock * kKStride];
-    __shared__ __align__(16) __nv_bfloat16 Vs[kBlock * kD];
-    __shared__ __align__(16) float Qs[G * kD];
-    __shared__ float Ps[G * kBlock];
-    __shared__ float m_s[G], l_s[G], scale_s[G];
-
-    const int split = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-    const int splits = gridDim.x;
-    const int tid = threadIdx.x;
-    const int L = kv_len[n];
-    const bool len_ok = L >= 1 && L <= max_pages * kBlock;
-    if (!len_ok) flag_status(status, kStatusBadData);
-    const int c = len_ok ? (L - 1) / kBlock : 0;
-    const long long sel_row = (long long)n * Hkv + h;
-    int n_sel = cnt[sel_row];
-    if (n_sel < 0 || n_sel > min(K, c)) { flag_status(status, kStatusBadData); n_sel = max(0, min(n_sel, min(K, c))); }
-    const int t0 = split * kBps;
-    const int t1 = len_ok ? min(t0 + kBps, n_sel + 1) : t0;
-
-    for (int e = tid; e < G * kD; e += kThreads) {
-        const int g = e / kD, d = e % kD;
-        Qs[e] = __bfloat162float(q[((long long)n * Hq + h * G + g) * kD + d]) * sm_scale * kLog2e;
+struct ItemInfo {
+    int n, h, L, c, n_sel;
+    bool ok;
+};
+__device__ __forceinline__ ItemInfo item_info(const Params& p, int item, bool flag) {
+    ItemInfo r;
+    r.n = item / p.Hkv;
+    r.h = item % p.Hkv;
+    r.L = p.kv_len[r.n];
+    r.ok = r.L >= 1 && r.L <= p.max_pages * kBlock;
+    r.c = r.ok ? (r.L - 1) / kBlock : 0;
+    int n_sel = p.cnt[item];
+    const int hi = min(p.K, r.c);
+    if (n_sel < 0 || n_sel > hi) {
+        if (flag) flag_status(p.status, kStatusBadData);
+        n_sel = max(0, min(n_sel, hi));
     }
-    if (tid < G) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
-    float acc[ITEMS][2];
-#pragma unroll
-    for (int it = 0; it < ITEMS; ++it) acc[it][0] = acc[it][1] = 0.f;
+    r.n_sel = n_sel;
+    if (!r.ok && flag) flag_status(p.status, kStatusBadData);
+    return r;
+}
 
-    for (int t = t0; t < t1; ++t) {
-        const bool cur = (t == n_sel);
-        const int j = cur ? c : idx[sel_row * K + t];
-        int page = -1;
-        if (j >= 0 && (cur || j < c) && j < max_pages) page = page_table[(long long)n * max_pages + j];
-        const bool ok = page >= 0 && page < num_pages;
-        if (!ok) flag_status(status, kStatusBadData);
-        const int nvalid = cur ? L - c * kBlock : kBlock;
-        const float bias = cur ? 0.f : log_gate[sel_row * K + t] * kLog2e;
-        __syncthreads();                       // previous block fully consumed
-        if (ok) {
-            const uint4* ksrc = reinterpret_cast<const uint4*>(kc + ((long long)page * Hkv + h) * kBlock * kD);
-            const uint4* vsrc = reinterpret_cast<const uint4*>(vc + ((long long)page * Hkv + h) * kBlock * kD);
-            for (int e = tid; e < kBlock * kD / 8; e += kThreads) {
-                const int r = e / (kD / 8), cc = e % (kD / 8);
-                uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-                if (r < nvalid) { kv = __ldg(ksrc + e); vv = __ldg(vsrc + e); }
-                *reinterpret_cast<uint4*>(Ks + r * kKStride + cc * 8) = kv;
-                *reinterpret_cast<uint4*>(Vs + r * kD + cc * 8) = vv;
-            }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, rows 8..15 zero: only a0a1 / a4a5 given) * B (16x8 bf16)
+__device__ __forceinline__ void mma_rows8(float (&d)[4], uint32_t a01, uint32_t a45, uint32_t b01, uint32_t b23) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a01), "r"(0u), "r"(a45), "r"(0u), "r"(b01), "r"(b23));
+}
+
+// Byte offset of 16-byte chunk `c` (0..15 over the 128 dims) of row `r` in a
+// tile stored as two 64-row x 128-byte boxes with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+    return (uint32_t)(c >> 3) * kBoxBytes + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* mo = reinterpret_cast<float*>(smem + kOffMo);
+    float* ml = reinterpret_cast<float*>(smem + kOffMl);
+    float2* meta = reinterpret_cast<float2*>(smem + kOffMeta);   // (bias log2 units, valid keys)
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* empty = full + kStages;
+    int* abort_flag = reinterpret_cast<int*>(empty + kStages);
+    volatile int* abort = abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        __syncthreads();
-        if (!ok) continue;
-        // logits (log2 domain) for every (head, key) of the block
-        for (int e = tid; e < G * kBlock; e += kThreads) {
-            const int g = e / kBlock, u = e % kBlock;
-            const uint4* kr = reinterpret_cast<const uint4*>(Ks + u * kKStride);
-            const float4* qr = reinterpret_cast<const float4*>(Qs + g * kD);
-            float dot = 0.f;
-#pragma unroll
-            for (int cc = 0; cc < kD / 8; ++cc) {
-                const uint4 w = kr[cc];
-                const float4 qa = qr[2 * cc], qb = qr[2 * cc + 1];
-                float2 f;
-                f = bf16x2_to_f32(w.x); dot = fmaf(qa.x, f.x, dot); dot = fmaf(qa.y, f.y, dot);
-                f = bf16x2_to_f32(w.y); dot = fmaf(qa.z, f.x, dot); dot = fmaf(qa.w, f.y, dot);
-                f = bf16x2_to_f32(w.z); dot = fmaf(qb.x, f.x, dot); dot = fmaf(qb.y, f.y, dot);
-                f = bf16x2_to_f32(w.w); dot = fmaf(qb.z, f.x, dot); dot = fmaf(qb.w, f.y, dot);
-            }
-            Ps[e] = (u < nvalid) ? dot + bias : -INFINITY;
-        }
-        __syncthreads();
-        // online softmax update, one warp per head
-        for (int g = tid >> 5; g < G; g += kThreads / 32) {
-            const int lane = tid & 31;
-            const float a = Ps[g * kBlock + lane], b2 = Ps[g * kBlock + 32 + lane];
-            const float bm = warp_max(fmaxf(a, b2));
-            const float mo = m_s[g];
-            const float mn = fmaxf(mo, bm);
-            const float pa = exp2f(a - mn), pb = exp2f(b2 - mn);
-            Ps[g * kBlock + lane] = pa;
-            Ps[g * kBlock + 32 + lane] = pb;
-            const float ps = warp_sum(pa + pb);
-            if (lane == 0) {
-                const float sc = exp2f(mo - mn);
-                scale_s[g] = sc;
-                l_s[g] = l_s[g] * sc + ps;
-                m_s[g] = mn;
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int it = 0; it < ITEMS; ++it) {
-            const int e = tid + it * kThreads;
-            if (e < G * 64) {
-                const int g = e / 64, dp = e % 64;
-                const float sc = scale_s[g];
-                float a0 = acc[it][0] * sc, a1 = acc[it][1] * sc;
-                const float* pr = Ps + g * kBlock;
-                const uint32_t* vcol = reinterpret_cast<const uint32_t*>(Vs) + dp;
-#pragma unroll 8
-                for (int u = 0; u < kBlock; ++u) {
-                    const float p = pr[u];
-                    const float2 f = bf16x2_to_f32(vcol[u * (kD / 2)]);
-                    a0 = fmaf(p, f.x, a0);
-                    a1 = fmaf(p, f.y, a1);
-                }
-                acc[it][0] = a0;
-                acc[it][1] = a1;
-            }
-        }
+        *abort_flag = 0;
+        fence_barrier_init();
     }
     __syncthreads();
-#pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
-        const int e = tid + it * kThreads;
-        if (e < G * 64) {
-            const int g = e / 64, dp = e % 64;
-            float* dst = part.o + (((long long)n * Hq + h * G + g) * splits + split) * kD + 2 * dp;
-            dst[0] = acc[it][0];
-            dst[1] = acc[it][1];
+
+    const long long v0 = slot_begin(blockIdx.x, p.V, p.grid), v1 = slot_begin(blockIdx.x + 1, p.V, p.grid);
+    const int Kp1 = p.K + 1;
+
+    if (warp == kWarps) {
+        // ----------------------------------------------------------- producer
+        // The 32 lanes resolve 32 block slots at a time (selection entry, page,
+        // gate: dependent loads, done in parallel); lane 0 then issues the
+        // copies of the kept ones in slot order.
+        if (lane == 0) {
+            prefetch_tensormap(&map_k);
+            prefetch_tensormap(&map_v);
         }
+        uint32_t it = 0;
+        bool ok_run = true;
+        for (long long base = v0; base < v1 && ok_run; base += 32) {
+            const long long v = base + lane;
+            bool use = false;
+            int row0 = -1;
+            float bias = 0.f, nvalid = 0.f;
+            if (v < v1) {
+                const int item = (int)(v / Kp1), t = (int)(v % Kp1);
+                const ItemInfo inf = item_info(p, item, true);
+                if (inf.ok && t <= inf.n_sel) {
+                    use = true;
+                    const bool cur = (t == inf.n_sel);
+                    const long long srow = (long long)item * p.K + t;
+                    const int j = cur ? inf.c : p.idx[srow];
+                    int page = -1;
+                    if (j >= 0 && (cur || j < inf.c) && j < p.max_pages)
+                        page = p.page_table[(long long)inf.n * p.max_pages + j];
+                    const bool ok = page >= 0 && page < p.num_pages;
+                    if (!ok) flag_status(p.status, kStatusBadData);
+                    bias = cur ? 0.f : p.log_gate[srow] * kLog2e;
+                    nvalid = ok ? (float)(cur ? inf.L - inf.c * kBlock : kBlock) : 0.f;
+                    row0 = ok ? (page * p.Hkv + inf.h) * kBlock : -1;   // < 2^31 (checked on the host)
+                }
+            }
+            unsigned todo = __ballot_sync(0xffffffffu, use);
+            while (todo) {
+                const int b = __ffs(todo) - 1;
+                todo &= todo - 1;
+                const int rb = __shfl_sync(0xffffffffu, row0, b);
+                const float bb = __shfl_sync(0xffffffffu, bias, b);
+                const float nb = __shfl_sync(0xffffffffu, nvalid, b);
+                if (lane == 0) {
+                    const int st = it % kStages;
+                    if (!mbar_wait(&empty[st], ((it / kStages) & 1) ^ 1, abort, p.status)) {
+                        ok_run = false;
+                    } else {
+                        meta[st] = make_float2(bb, nb);
+                        if (rb >= 0) {
+                            mbar_expect_tx(&full[st], kStageBytes);
+                            uint8_t* dst = smem + st * kStageBytes;
+                            for (int a = 0; a < 2; ++a) {
+                                tma_load_3d(dst + a * kBoxBytes, &map_k, &full[st], a * 64, 0, rb);
+                                tma_load_3d(dst + kTileBytes + a * kBoxBytes, &map_v, &full[st], a * 64, 0, rb);
+                            }
+                        } else {
+                            mbar_arrive(&full[st]);
+                        }
+                        ++it;
+                    }
+                }
+                ok_run = __shfl_sync(0xffffffffu, ok_run, 0);
+                if (!ok_run) break;
+            }
+        }
+        if (lane == 0 && *abort) {       // let the copies in flight land before the CTA exits
+            volatile int no_abort = 0;
+            const uint32_t lo = it > (uint32_t)kStages ? it - kStages : 0;
+            for (uint32_t k = lo; k < it; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, &no_abort, nullptr);
+        }
+        return;   // the producer takes no part in the consumers' named barrier
     }
-    if (tid < G) {
-        float* ml = part.ml + (((long long)n * Hq + h * G + tid) * splits + split) * 2;
-        ml[0] = m_s[tid];
-        ml[1] = l_s[tid];
+
+    // -------------------------------------------------------------- consumers
+    const int grp = lane >> 2, tig = lane & 3;     // mma fragment coordinates: row (head), column pair
+    const uint32_t s_base = smem_u32(smem);
+    uint32_t qa[8][2];          // Q as A fragments: 8 k-steps x (dims 2tig.., 8+2tig..) of head grp
+    float o[16][4];             // O accumulators: 16 n-tiles of 8 dims (rows 8..15 stay 0)
+    float m = -INFINITY, l = 0.f;   // this thread's head: running max (log2) and its partial sum
+    uint32_t blk = 0;           // blocks of this CTA's stream seen so far
+    int cur_item = -1;
+    ItemInfo inf{};
+    bool dead = false;
+
+    auto flush = [&]() {
+        // row sum over the quad, then every warp's state to shared memory
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+            *reinterpret_cast<float2*>(mo + (warp * 8 + grp) * kD + 8 * nt + 2 * tig) = make_float2(o[nt][0], o[nt][1]);
+        if (tig == 0) {
+            ml[(warp * 8 + grp) * 2] = m;
+            ml[(warp * 8 + grp) * 2 + 1] = l;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+        const int slot = (int)blockIdx.x - cta_of((long long)cur_item * Kp1, p.V, p.grid);
+        for (int e = threadIdx.x; e < p.G * kD; e += kWarps * 32) {
+            const int g = e / kD, d = e % kD;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, ml[(w * 8 + g) * 2]);
+            float acc = 0.f, L = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    const float mw = ml[(w * 8 + g) * 2];
+                    const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                    acc = fmaf(mo[(w * 8 + g) * kD + d], f, acc);
+                    L = fmaf(ml[(w * 8 + g) * 2 + 1], f, L);
+                }
+            }
+            const long long row = ((long long)inf.n * p.Hq + inf.h * p.G + g) * p.nslot + slot;
+            p.part_o[row * kD + d] = acc;
+            if (d == 0) {
+                p.part_ml[row * 2] = M;
+                p.part_ml[row * 2 + 1] = L;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+    };
+
+    for (long long v = v0; v < v1; ++v) {
+        const int item = (int)(v / Kp1), t = (int)(v % Kp1);
+        if (item != cur_item) {
+            if (cur_item >= 0) flush();
+            cur_item = item;
+            inf = item_info(p, item, false);
+            const bool real = grp < p.G;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                p.q + ((long long)inf.n * p.Hq + inf.h * p.G + (real ? grp : 0)) * kD);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                qa[kk][0] = real ? __ldg(qrow + 8 * kk + tig) : 0u;
+                qa[kk][1] = real ? __ldg(qrow + 8 * kk + 4 + tig) : 0u;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+            m = -INFINITY;
+            l = 0.f;
+        }
+        if (!inf.ok || t > inf.n_sel) continue;
+        const uint32_t b = blk++;
+        if (b % kWarps != (uint32_t)warp || dead) continue;      // another warp's block
+        const int st = b % kStages;
+        if (!mbar_wait_warp(&full[st], (b / kStages) & 1, abort, p.status)) {
+            dead = true;              // keep walking the slots so the flush barriers still meet
+            continue;
+        }
+        const float2 md = meta[st];
+        const int nvalid = (int)md.y;
+        if (nvalid > 0) {
+            const uint32_t kt = s_base + st * kStageBytes, vt = kt + kTileBytes;
+            // S = Q K^T: n-tile nt = keys 8nt..8nt+7; ldmatrix.x4 gives B fragments of two n-tiles
+            float s[8][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    const int key = 16 * np + 8 * (lane >> 4) + (lane & 7);
+                    const int chunk = 2 * kk + ((lane >> 3) & 1);
+                    uint32_t bf[4];
+                    ldsm_x4(kt + tile_off(key, chunk), bf);
+                    mma_rows8(s[2 * np], qa[kk][0], qa[kk][1], bf[0], bf[1]);
+                    mma_rows8(s[2 * np + 1], qa[kk][0], qa[kk][1], bf[2], bf[3]);
+                }
+            }
+            // online softmax for head grp over keys 8nt + 2tig + {0, 1}
+            float bm = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int key = 8 * nt + 2 * tig + e;
+                    const float x = key < nvalid ? fmaf(s[nt][e], p.qscale, md.x) : -INFINITY;
+                    s[nt][e] = x;
+                    bm = fmaxf(bm, x);
+                }
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+            const float mn = fmaxf(m, bm);
+            const float sc = mn == -INFINITY ? 1.f : exp2f(m - mn);
+            m = mn;
+            uint32_t pa[8];             // P as A fragments: n-tile nt -> keys 8nt + 2tig..
+            float ls = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const float p0 = mn == -INFINITY ? 0.f : exp2f(s[nt][0] - mn);
+                const float p1 = mn == -INFINITY ? 0.f : exp2f(s[nt][1] - mn);
+                ls += p0 + p1;
+                pa[nt] = pack_bf16x2(p0, p1);
+            }
+            l = fmaf(l, sc, ls);
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][0] *= sc;
+                o[nt][1] *= sc;
+            }
+            if (nvalid < kBlock) {
+                // rows past the sequence end (the current block) are zeroed: their p
+                // is 0, but whatever the page holds there must not reach O as 0 * NaN
+                uint8_t* vrow = smem + st * kStageBytes + kTileBytes;
+                for (int e = nvalid * 16 + lane; e < kBlock * 16; e += 32)
+                    *reinterpret_cast<uint4*>(vrow + tile_off(e >> 4, e & 15)) = make_uint4(0u, 0u, 0u, 0u);
+                fence_proxy_async_smem();     // ordered before the stage's next TMA refill
+                __syncwarp();
+            }
+            // O += P V: k-step kk = keys 16kk..16kk+15; ldmatrix.x4.trans gives B of two n-tiles
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int np = 0; np < 8; ++np) {
+                    const int key = 16 * kk + 8 * ((lane >> 3) & 1) + (lane & 7);
+                    const int chunk = 2 * np + (lane >> 4);
+                    uint32_t bf[4];
+                    ldsm_x4_t(vt + tile_off(key, chunk), bf);
+                    mma_rows8(o[2 * np], pa[2 * kk], pa[2 * kk + 1], bf[0], bf[1]);
+                    mma_rows8(o[2 * np + 1], pa[2 * kk], pa[2 * kk + 1], bf[2], bf[3]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
+    if (cur_item >= 0) flush();
 }
 
 __global__ void __launch_bounds__(kD)
-decode_combine_kernel(Part part, int splits, int Hq, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, int nslot, int Hq, int Hkv,
+                      int G, int K, long long V, int grid, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
     const long long row = blockIdx.x;          // n * Hq + hq
     const int d = threadIdx.x;
-    const float* ml = part.ml + row * splits * 2;
+    const long long n = row / Hq;
+    const int hq = (int)(row % Hq);
+    const long long item = n * Hkv + hq / G;
+    const long long s0 = item * (K + 1);
+    const int nsl = cta_of(s0 + K, V, grid) - cta_of(s0, V, grid) + 1;
+    const float* ml = part_ml + row * nslot * 2;
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
+    for (int s = 0; s < nsl; ++s) M = fmaxf(M, ml[2 * s]);
     float Lsum = 0.f, acc = 0.f;
     if (M != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float w = exp2f(ml[2 * s] - M);     // 0 for empty splits (m = -inf)
+        for (int s = 0; s < nsl; ++s) {
+            const float w = exp2f(ml[2 * s] - M);     // 0 for empty partials (m = -inf)
             Lsum = fmaf(ml[2 * s + 1], w, Lsum);
-            acc = fmaf(part.o[(row * splits + s) * kD + d], w, acc);
+            acc = fmaf(part_o[(row * nslot + s) * kD + d], w, acc);
         }
     }
     o[row * kD + d] = __float2bfloat16_rn(acc / Lsum);
     if (lse != nullptr && d == 0) lse[row] = (M + log2f(Lsum)) * kLn2;
 }
 
-template <int G>
-cudaError_t go(const DecodeArgs& a, Part part, cudaStream_t st) {
-    const int splits = num_splits(a.K);
-    dim3 grid(splits, a.Hkv, a.N);
-    decode_split_kernel<G><<<grid, kThreads, 0, st>>>(
-        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k_cache, (const __nv_bfloat16*)a.v_cache,
-        a.num_pages, a.page_table, a.max_pages, a.kv_len, a.Hq, a.Hkv, a.K, a.idx, a.cnt,
-        a.log_gate, a.sm_scale, part, a.status);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    decode_combine_kernel<<<a.N * a.Hq, kD, 0, st>>>(part, splits, a.Hq, (__nv_bfloat16*)a.o, a.lse);
-    count_launches(2);
-    return cudaGetLastError();
+struct Layout {
+    long long V;
+    int grid, nslot;
+};
+Layout layout(int N, int Hkv, int K) {
+    Layout r;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    r.V = (long long)N * Hkv * (K + 1);
+    r.grid = (int)(r.V < sms ? r.V : sms);
+    if (r.grid < 1) r.grid = 1;
+    const long long mn = r.V / r.grid;                       // shortest CTA range
+    const long long span = (K + 1 + mn - 1) / mn + 1;        // CTAs one item's slots can touch
+    r.nslot = (int)(span < r.grid ? span : r.grid);
+    return r;
 }
 
 }  // namespace
 
 size_t decode_workspace(int N, int Hq, int Hkv, int D, int K) {
-    (void)Hkv; (void)D;
-    const size_t per = (size_t)N * Hq * num_splits(K);
+    (void)D;
+    const Layout lay = layout(N, Hkv, K);
+    const size_t per = (size_t)N * Hq * lay.nslot;
     return sizeof(float) * (per * kD + per * 2);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t st) {
-    Part part = carve(workspace, a.N, a.Hq, a.K);
-    switch (a.Hq / a.Hkv) {
-        case 1: return go<1>(a, part, st);
-        case 2: return go<2>(a, part, st);
-        case 4: return go<4>(a, part, st);
-        case 5: return go<5>(a, part, st);
-        case 8: return go<8>(a, part, st);
-        default: return cudaErrorInvalidValue;
-    }
+    const int G = a.Hq / a.Hkv;
+    if (G < 1 || G > 8 || a.Hq % a.Hkv) return cudaErrorInvalidValue;
+    const long long cache_rows = (long long)a.num_pages * a.Hkv * kBlock;
+    if (cache_rows > 0x7fffffffLL) return cudaErrorInvalidValue;   // TMA row coordinates are int32
+    const Layout lay = layout(a.N, a.Hkv, a.K);
+    float* part_o = static_cast<float*>(workspace);
+    float* part_ml = part_o + (size_t)a.N * a.Hq * lay.nslot * kD;
+    CUtensorMap mk, mv;
+    if (!make_head_map(&mk, a.k_cache, cache_rows, 1, kD) || !make_head_map(&mv, a.v_cache, cache_rows, 1, kD))
+        return cudaErrorInvalidValue;
+    Params p;
+    p.q = (const __nv_bfloat16*)a.q;
+    p.num_pages = a.num_pages;
+    p.page_table = a.page_table;
+    p.max_pages = a.max_pages;
+    p.kv_len = a.kv_len;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.G = G;
+    p.K = a.K;
+    p.idx = a.idx;
+    p.cnt = a.cnt;
+    p.log_gate = a.log_gate;
+    p.qscale = a.sm_scale * kLog2e;
+    p.V = lay.V;
+    p.grid = lay.grid;
+    p.nslot = lay.nslot;
+    p.part_o = part_o;
+    p.part_ml = part_ml;
+    p.status = a.status;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
+    decode_kernel<<<lay.grid, kThreads, kSmem, st>>>(mk, mv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    decode_combine_kernel<<<a.N * a.Hq, kD, 0, st>>>(part_o, part_ml, lay.nslot, a.Hq, a.Hkv, G, a.K, lay.V,
+                                                      lay.grid, (__nv_bfloat16*)a.o, a.lse);
+    count_launches(2);
+    return cudaGetLastError();
 }
 
 }  // namespace sas

@@ -11,10 +11,11 @@
 //
 // Two tensor-core kernels, no floating-point atomics on dq/dk/dv:
 //  * dq_kernel (query-stationary, like the forward): item = (b, h, i, head
-//    group), up to two 128-row Q tiles (2 heads x 64 rows each) sharing each
-//    kept K/V block. Per block: S = Q K^T and dP = dO V^T into TMEM, dS to a
-//    swizzled shared-memory tile, dQ += dS K accumulated in TMEM across the
-//    item. Also the per-block gate gradients (warp sums of dS).
+//    pair), one 128-row Q tile (2 heads x 64 rows) whose Q and dO stay in
+//    TMEM for the item. Per kept block: S = Q K^T and dP = dO V^T (A from
+//    TMEM) into one of two TMEM buffers, dS to a swizzled shared-memory tile,
+//    dQ += dS K accumulated in TMEM across the item. Also the per-block gate
+//    gradients (warp sums of dS).
 //  * dkv_kernel (key-stationary): item = (b, h, j); walks the query blocks
 //    that attend block j (its own block and every block that kept it, from a
 //    reverse index), one Q tile per step, and accumulates dV^T = sum dO^T P
@@ -53,7 +54,7 @@ constexpr uint32_t kHi = sm100::sdesc_hi(1024);   // high descriptor word: 8-row
 
 // ------------------------------------------------------------------ shared
 struct Params {
-    int B, S, Hq, Hkv, G, K, NQB, ntg, n_items, ntile;
+    int B, S, Hq, Hkv, G, K, NQB, n_items, ntile;
     const int32_t* idx;
     const int32_t* cnt;
     const float* log_gate;
@@ -111,39 +112,48 @@ __device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32
 // ===================================================================== dq
 namespace dqk {
 
-constexpr uint32_t kOffQ = 0;                      // 2 Q tiles
-constexpr uint32_t kOffO = 2 * kTile;              // 2 dO tiles
-constexpr uint32_t kOffKV = 4 * kTile;             // 2 stages x (K block, V block)
-constexpr int kNS = 2;
-constexpr uint32_t kStage = 2 * kBlk;
-constexpr uint32_t kOffDS = kOffKV + kNS * kStage;        // 2 dS tiles
-constexpr uint32_t kOffBar = kOffDS + 2 * kRowTile;      // 224 KB
+// One 128-row Q tile (two heads x 64 rows of query block i) per item; Q and
+// dO stay in TMEM for the whole item (A operands of S = Q K^T, dP = dO V^T),
+// the kept K/V blocks stream through a 4-stage ring.
+constexpr int kNS = 4;
+constexpr uint32_t kStage = 2 * kBlk;                      // K block, V block
+constexpr uint32_t kOffKV = 0;
+constexpr uint32_t kOffQs = kOffKV + kNS * kStage;         // staging: Q tile, dO tile (TMA -> TMEM)
+constexpr uint32_t kOffDS = kOffQs + 2 * kTile;            // 2 dS tiles (one per warpgroup)
+constexpr uint32_t kOffBar = kOffDS + 2 * kRowTile;        // 224 KB
 constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
+// TMEM columns
+constexpr uint32_t kTmQ = 0, kTmO = 64, kTmS = 128, kTmDQ = 384;   // S/dP buffer u at kTmS + 128 u (S, dP + 64)
+
+// warps: 0 TMA; 2-5 / 6-9 softmax warpgroups 0 / 1 (warpgroup u takes the
+// blocks of odd / even position in the CTA's block stream); issuing warps
+// 1, 10: S of stream parity 0 / 1; 11, 12: dP of parity 0 / 1; 13: dQ
+constexpr int kThreadsDq = 448;
 
 struct Bars {
-    uint64_t qd_full, qd_empty;
+    uint64_t qs_full, qs_empty, qt_full, qt_free;       // Q/dO staging full/empty, TMEM copy full/free
     uint64_t k_full[kNS], v_full[kNS], kv_empty[kNS];
-    uint64_t s_full[2], tm_free[2], ds_full[2], ds_empty[2], dq_full[2], dq_empty[2];
-    uint64_t drain[4];
+    uint64_t s_full[2], tm_free[2], ds_full[2], ds_empty[2];
+    uint64_t dq_full, dq_empty;
+    uint64_t drain[5];
     uint32_t tmem_base;
     int abort;
 };
 
 struct Item {
-    int b, h, i, tg, nt, c, nb;
-    long long row;
+    int b, h, i, t, c, nb;
+    long long row;     // selection row (b, h, i)
 };
 
 __device__ __forceinline__ Item item_of(const Params& p, int id) {
     Item it;
-    const int per_i = p.B * p.Hkv * p.ntg;
-    it.i = p.NQB - 1 - id / per_i;
+    const int per_i = p.B * p.Hkv * p.ntile;
+    it.i = p.NQB - 1 - id / per_i;          // longest items first
     int r = id % per_i;
-    it.tg = r % p.ntg;
-    r /= p.ntg;
+    it.t = r % p.ntile;
+    r /= p.ntile;
     it.h = r % p.Hkv;
     it.b = r / p.Hkv;
-    it.nt = (4 * it.tg + 2 < p.G) ? 2 : 1;
     it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
     it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));
     it.nb = it.c + 1;
@@ -173,7 +183,7 @@ __device__ __forceinline__ Blk block_at(const Params& p, const Item& it, int k) 
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsDq, 1)
 dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
           const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -182,22 +192,24 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &bars->abort;
     if (threadIdx.x == 0) {
-        mbar_init(&bars->qd_full, 1);
-        mbar_init(&bars->qd_empty, 4);                  // one arrival per issuing warp
+        mbar_init(&bars->qs_full, 1);
+        mbar_init(&bars->qs_empty, 256);                 // both warpgroups copied their half
+        mbar_init(&bars->qt_full, 256);
+        mbar_init(&bars->qt_free, 4);                    // the four S / dP warps
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 4);
+            mbar_init(&bars->kv_empty[s], 3);            // S, dP and dQ warps
         }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(&bars->s_full[t], 2);             // S and dP come from two warps
-            mbar_init(&bars->tm_free[t], 128);
-            mbar_init(&bars->ds_full[t], 128);
-            mbar_init(&bars->ds_empty[t], 1);
-            mbar_init(&bars->dq_full[t], 1);
-            mbar_init(&bars->dq_empty[t], 128);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&bars->s_full[u], 2);              // S and dP warps
+            mbar_init(&bars->tm_free[u], 128);
+            mbar_init(&bars->ds_full[u], 128);
+            mbar_init(&bars->ds_empty[u], 1);
         }
-        for (int w = 0; w < 4; ++w) mbar_init(&bars->drain[w], 1);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_empty, 256);
+        for (int w = 0; w < 5; ++w) mbar_init(&bars->drain[w], 1);
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -209,33 +221,42 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t sQ = smem_u32(smem + kOffQ), sO = smem_u32(smem + kOffO), sKV = smem_u32(smem + kOffKV);
-    const uint32_t sDS = smem_u32(smem + kOffDS);
+    const uint32_t s_base = smem_u32(smem);
 
     if (warp == 0) {
+        // ---------------------------------------------------------------- TMA
         if (lane == 0) {
-            uint32_t kv_it = 0, q_it = 0;
-            int last_it[kNS] = {-1, -1};
-            bool q_issued = false;
-            for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x) {
+            uint32_t kb = 0, qn = 0;
+            int last_kv[kNS] = {-1, -1, -1, -1};
+            bool q_pending = false;
+            // Q/dO tile of item `id` into the staging buffer (once the previous one
+            // has been copied to TMEM)
+            auto load_qd = [&](int id) -> bool {
                 const Item it = item_of(p, id);
-                if (!mbar_wait(&bars->qd_empty, (q_it & 1) ^ 1, abort, p.status)) break;
-                mbar_expect_tx(&bars->qd_full, (uint32_t)it.nt * 8 * kBox);
-                for (int t = 0; t < it.nt; ++t)
-                    for (int s = 0; s < 2; ++s) {
-                        const int slot = 4 * it.tg + 2 * t + s;
-                        const int hq = it.h * p.G + (slot < p.G ? slot : 0);
-                        for (int a = 0; a < 2; ++a) {
-                            const uint32_t off = t * kTile + a * kTileAtom + s * kBox;
-                            tma_load_3d(smem + kOffQ + off, &map_q, &bars->qd_full, a * 64, hq, it.b * p.S + it.i * 64);
-                            tma_load_3d(smem + kOffO + off, &map_do, &bars->qd_full, a * 64, hq, it.b * p.S + it.i * 64);
-                        }
+                if (!mbar_wait(&bars->qs_empty, (qn & 1) ^ 1, abort, p.status)) return false;
+                mbar_expect_tx(&bars->qs_full, 8 * kBox);
+                for (int s = 0; s < 2; ++s) {
+                    const int slot = 2 * it.t + s;
+                    const int hq = it.h * p.G + (slot < p.G ? slot : 0);
+                    for (int a = 0; a < 2; ++a) {
+                        const uint32_t off = a * kTileAtom + s * kBox;
+                        tma_load_3d(smem + kOffQs + off, &map_q, &bars->qs_full, a * 64, hq, it.b * p.S + it.i * 64);
+                        tma_load_3d(smem + kOffQs + kTile + off, &map_do, &bars->qs_full, a * 64, hq,
+                                    it.b * p.S + it.i * 64);
                     }
-                q_issued = true;
-                ++q_it;
-                for (int k = 0; k < it.nb; ++k, ++kv_it) {
-                    const int st = kv_it % kNS;
-                    if (!mbar_wait(&bars->kv_empty[st], ((kv_it / kNS) & 1) ^ 1, abort, p.status)) break;
+                }
+                ++qn;
+                q_pending = true;
+                return true;
+            };
+            bool ok = blockIdx.x >= p.n_items || load_qd(blockIdx.x);
+            for (int id = blockIdx.x; id < p.n_items && ok && !*abort; id += gridDim.x) {
+                const Item it = item_of(p, id);
+                const int nxt = id + gridDim.x;
+                const int k_next = min(1, it.nb - 1);   // the next item's Q/dO goes out after this block
+                for (int k = 0; k < it.nb && ok; ++k, ++kb) {
+                    const int st = kb % kNS;
+                    if (!(ok = mbar_wait(&bars->kv_empty[st], ((kb / kNS) & 1) ^ 1, abort, p.status))) break;
                     const Blk bk = block_at(p, it, k);
                     if (!bk.valid) flag_status(p.status, kStatusBadData);
                     mbar_expect_tx(&bars->k_full[st], 2 * kBox);
@@ -246,131 +267,150 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     for (int a = 0; a < 2; ++a)
                         tma_load_3d(smem + kOffKV + st * kStage + kBlk + a * kBlkAtom, &map_v, &bars->v_full[st],
                                     a * 64, it.h, it.b * p.S + bk.j * 64);
-                    last_it[st] = (int)kv_it;
+                    last_kv[st] = (int)kb;
+                    if (k == k_next && nxt < p.n_items) ok = load_qd(nxt);
                 }
             }
-            if (*abort) {
+            if (*abort) {           // let every copy in flight land before the CTA exits
                 volatile int no_abort = 0;
                 for (int s = 0; s < kNS; ++s)
-                    if (last_it[s] >= 0) {
-                        const uint32_t par = ((uint32_t)last_it[s] / kNS) & 1;
+                    if (last_kv[s] >= 0) {
+                        const uint32_t par = ((uint32_t)last_kv[s] / kNS) & 1;
                         mbar_wait(&bars->k_full[s], par, &no_abort, nullptr);
                         mbar_wait(&bars->v_full[s], par, &no_abort, nullptr);
                     }
-                if (q_issued) mbar_wait(&bars->qd_full, (q_it - 1) & 1, &no_abort, nullptr);
+                if (q_pending) mbar_wait(&bars->qs_full, (qn - 1) & 1, &no_abort, nullptr);
             }
         }
-    } else if (is_issuer_warp(warp)) {
-        // slot 0 / 1: S and dQ of tile 0 / 1 (reads Q, K, dS); slot 2 / 3: dP of
-        // tile 0 / 1 (reads dO, V). The whole warp runs the loop, one lane issues.
-        const int slot = issuer_slot(warp);
-        const int t = slot & 1;                         // the Q tile this warp issues for
-        const bool sq = slot < 2;
-        const uint32_t id_s = idesc_bf16(128, 64, false, false);
-        const uint32_t id_dq = idesc_bf16(128, kD, false, true);
-        const uint32_t a_lo = sdesc_lo((sq ? sQ : sO) + t * kTile, 16);
-        const uint32_t d_sp = tmem + 256 * t + (sq ? 0u : 64u);
-        const uint32_t b_off = sq ? 0u : kBlk;          // K or V inside a stage
-        uint32_t kv_it = 0, q_it = 0, ds_it = 0, de_it = 0, sdp_n = 0;
+    } else if (warp == 1 || warp >= 10) {
+        // ----------------------------------------------------- issuing warps
+        const int slot = warp == 1 ? 0 : warp - 9;      // 0, 1: S parity 0/1; 2, 3: dP parity 0/1; 4: dQ
+        uint32_t kb = 0, qn = 0;
         bool ok = true;
-        // S (or dP) of this tile for the block in stage st, once the warpgroup has
-        // read the previous one out of TMEM
-        auto issue_sp = [&](int st) -> bool {
-            if (sdp_n > 0 && !mbar_wait_warp(&bars->tm_free[t], (sdp_n - 1) & 1, abort, p.status)) return false;
-            ++sdp_n;
-            tc_fence_after();
-            const uint32_t b_lo = sdesc_lo(sKV + st * kStage + b_off, 16);
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                mma_ss_e(d_sp, a_lo + (ao >> 4), kHi, b_lo + (bo >> 4), kHi, id_s, kk > 0);
-            }
-            mma_commit_e(&bars->s_full[t]);
-            return true;
-        };
-        auto wait_stage = [&](uint32_t n) -> bool {
-            const int st = n % kNS;
-            return mbar_wait_warp(sq ? &bars->k_full[st] : &bars->v_full[st], (n / kNS) & 1, abort, p.status);
-        };
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
-            const Item it = item_of(p, id);
-            if (t >= it.nt) {                       // tile 1 idle: tile 0's warps arrive for it
-                kv_it += it.nb;
-                ++q_it;
-                continue;
-            }
-            const int owe = (it.nt == 1) ? 2 : 1;   // arrivals owed to the shared stage barriers
-            if (!(ok = mbar_wait_warp(&bars->qd_full, q_it & 1, abort, p.status))) break;
-            ++q_it;
-            if (!(ok = wait_stage(kv_it) && issue_sp(kv_it % kNS))) break;
-            if (it.nb == 1)
-                for (int c = 0; c < owe; ++c) mma_commit_e(&bars->qd_empty);
-            for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
-                const int st = kv_it % kNS;
-                const bool more = k + 1 < it.nb;
-                if (more) {                         // one block ahead
-                    if (!(ok = wait_stage(kv_it + 1) && issue_sp((kv_it + 1) % kNS))) break;
-                    if (k + 2 == it.nb)             // that was the last MMA reading this Q (dO) tile
-                        for (int c = 0; c < owe; ++c) mma_commit_e(&bars->qd_empty);
-                }
-                if (sq) {
-                    if (!(ok = mbar_wait_warp(&bars->ds_full[t], ds_it & 1, abort, p.status))) break;
-                    ++ds_it;
-                    if (k == 0) {
-                        if (!(ok = mbar_wait_warp(&bars->dq_empty[t], (de_it & 1) ^ 1, abort, p.status))) break;
-                        ++de_it;
-                    }
+        if (slot < 4) {
+            const int u = slot & 1;
+            const bool is_s = slot < 2;
+            const uint32_t id_s = idesc_bf16(128, 64, false, false);
+            const uint32_t a_tm = tmem + (is_s ? kTmQ : kTmO);
+            const uint32_t d_tm = tmem + kTmS + 128 * u + (is_s ? 0u : 64u);
+            const uint32_t b_off = is_s ? 0u : kBlk;
+            uint32_t n_mine = 0;
+            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
+                const Item it = item_of(p, id);
+                // this item's Q and dO are in TMEM
+                if (!(ok = mbar_wait_warp(&bars->qt_full, qn & 1, abort, p.status))) break;
+                tc_fence_after();
+                for (int k = 0; k < it.nb && ok; ++k, ++kb) {
+                    if ((kb & 1) != (uint32_t)u) continue;
+                    const int st = kb % kNS;
+                    uint64_t* fb = is_s ? &bars->k_full[st] : &bars->v_full[st];
+                    if (!(ok = mbar_wait_warp(fb, (kb / kNS) & 1, abort, p.status))) break;
+                    // warpgroup u has read its previous S / dP out of TMEM
+                    if (n_mine > 0 && !(ok = mbar_wait_warp(&bars->tm_free[u], (n_mine - 1) & 1, abort, p.status)))
+                        break;
+                    ++n_mine;
                     tc_fence_after();
-                    const uint32_t ds_lo = sdesc_lo(sDS + t * kRowTile, 16);         // K-major dS
-                    const uint32_t kt_lo = sdesc_lo(sKV + st * kStage, kBlkAtom);    // MN-major K
-                    const uint32_t acc0 = k > 0 ? 1u : 0u;
+                    const uint32_t b_lo = sdesc_lo(s_base + kOffKV + st * kStage + b_off, 16);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                        mma_ts_e(d_tm, a_tm + kk * 8, b_lo + (bo >> 4), kHi, id_s, kk > 0);
+                    }
+                    mma_commit_e(&bars->s_full[u]);
+                    mma_commit_e(&bars->kv_empty[st]);
+                }
+                if (!ok) break;
+                mma_commit_e(&bars->qt_free);           // done reading this item's Q / dO in TMEM
+            }
+        } else {
+            // dQ += dS K (SS: A = dS tile of the block's warpgroup, B = K MN-major)
+            const uint32_t id_dq = idesc_bf16(128, kD, false, true);
+            uint32_t ds_n[2] = {0, 0};
+            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
+                const Item it = item_of(p, id);
+                for (int k = 0; k < it.nb && ok; ++k, ++kb) {
+                    const int u = kb & 1, st = kb % kNS;
+                    if (!(ok = mbar_wait_warp(&bars->ds_full[u], ds_n[u] & 1, abort, p.status))) break;
+                    ++ds_n[u];
+                    // the previous item's dQ has been read out of TMEM
+                    if (k == 0 && !(ok = mbar_wait_warp(&bars->dq_empty, (qn & 1) ^ 1, abort, p.status))) break;
+                    tc_fence_after();
+                    const uint32_t ds_lo = sdesc_lo(s_base + kOffDS + u * kRowTile, 16);     // K-major dS
+                    const uint32_t kt_lo = sdesc_lo(s_base + kOffKV + st * kStage, kBlkAtom); // MN-major K
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ss_e(tmem + 256 * t + 128, ds_lo + ((kk * 32) >> 4), kHi, kt_lo + ((kk * 2048) >> 4), kHi,
-                                 id_dq, kk > 0 ? 1u : acc0);
-                    mma_commit_e(&bars->ds_empty[t]);
-                    if (!more) mma_commit_e(&bars->dq_full[t]);
+                        mma_ss_e(tmem + kTmDQ, ds_lo + ((kk * 32) >> 4), kHi, kt_lo + ((kk * 2048) >> 4), kHi, id_dq,
+                                 (k > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit_e(&bars->ds_empty[u]);
+                    mma_commit_e(&bars->kv_empty[st]);
+                    if (k + 1 == it.nb) mma_commit_e(&bars->dq_full);
                 }
-                for (int c = 0; c < owe; ++c) mma_commit_e(&bars->kv_empty[st]);
             }
         }
         mma_commit_e(&bars->drain[slot]);
         volatile int no_abort = 0;
         mbar_wait(&bars->drain[slot], 0, &no_abort, nullptr);
-    } else if (warp >= 2 && warp < 10) {
-        const int t = (warp - 2) >> 2;
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        const int u = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int slot_in_tile = row >> 6, r_in = row & 63;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_base + 256 * t;
+        const uint32_t tS = tmem + lane_base + kTmS + 128 * u;
         const uint32_t tP = tS + 64;
-        const uint32_t tQ = tS + 128;
-        uint8_t* ds_tile = smem + kOffDS + t * kRowTile;
-        uint32_t s_it = 0, q_it = 0, ds_n = 0;
-        for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
+        uint8_t* ds_tile = smem + kOffDS + u * kRowTile;
+        uint32_t kb = 0, qn = 0, s_it = 0, ds_n = 0;
+        bool ok = true;
+        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
             const Item it = item_of(p, id);
-            if (t >= it.nt) continue;
-            const int slot = 4 * it.tg + 2 * t + slot_in_tile;
+            // copy this warpgroup's half of the staged tile (0: Q, 1: dO) into TMEM once
+            // the S / dP warps are done with the previous item's
+            if (qn > 0 && !(ok = mbar_wait(&bars->qt_free, (qn - 1) & 1, abort, p.status))) break;
+            if (!(ok = mbar_wait(&bars->qs_full, qn & 1, abort, p.status))) break;
+            {
+                const uint8_t* src = smem + kOffQs + u * kTile;
+                const uint32_t dst = tmem + lane_base + (u == 0 ? kTmQ : kTmO);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {           // dims [64 a, 64 a + 64) -> 32 packed columns
+                    uint32_t v[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(src + a * kTileAtom + sw128_offset(row, c));
+                        v[4 * c] = w.x;
+                        v[4 * c + 1] = w.y;
+                        v[4 * c + 2] = w.z;
+                        v[4 * c + 3] = w.w;
+                    }
+                    tmem_st32(dst + 32 * a, v);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->qs_empty);
+            mbar_arrive(&bars->qt_full);
+
+            const int slot = 2 * it.t + slot_in_tile;
             const bool row_ok = slot < p.G;
             const int hq = it.h * p.G + (row_ok ? slot : 0);
             const long long lrow = ((long long)it.b * p.Hq + hq) * p.S + (long long)it.i * 64 + r_in;
             const float lse2 = p.lse[lrow] * kLog2e;
             const float drs = p.Dr[lrow] * p.sm_scale;
-            bool ok = true;
-            Blk nxt = block_at(p, it, 0);
-            for (int k = 0; k < it.nb; ++k) {
+            // this warpgroup's blocks: stream positions kb + k with (kb + k) % 2 == u
+            int k = (int)((u - (int)(kb & 1)) & 1);
+            Blk nxt;
+            if (k < it.nb) nxt = block_at(p, it, k);
+            for (; k < it.nb; k += 2) {
                 const Blk bk = nxt;
-                if (k + 1 < it.nb) nxt = block_at(p, it, k + 1);
-                if (!(ok = mbar_wait(&bars->s_full[t], s_it & 1, abort, p.status))) break;
+                if (k + 2 < it.nb) nxt = block_at(p, it, k + 2);
+                if (!(ok = mbar_wait(&bars->s_full[u], s_it & 1, abort, p.status))) break;
                 ++s_it;
                 tc_fence_after();
                 // log2 domain; rows of an absent head (or a bad block) get -inf: P = dS = 0
                 const float off = (row_ok && bk.valid) ? bk.bias2 - lse2 : -INFINITY;
                 float gs = 0.f;                           // sum of dS * sm_scale over the row's keys
-                // dQ of the previous step has finished reading the dS tile
-                if (ds_n > 0 && !(ok = mbar_wait(&bars->ds_empty[t], (ds_n - 1) & 1, abort, p.status))) break;
+                // dQ of this warpgroup's previous block has finished reading the dS tile
+                if (ds_n > 0 && !(ok = mbar_wait(&bars->ds_empty[u], (ds_n - 1) & 1, abort, p.status))) break;
                 ++ds_n;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {          // keys [32 hf, 32 hf + 32)
@@ -380,7 +420,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     tmem_wait_ld();
                     if (hf == 1) {
                         tc_fence_before();
-                        mbar_arrive(&bars->tm_free[t]);   // S/dP columns may be refilled
+                        mbar_arrive(&bars->tm_free[u]);   // S/dP columns may be refilled
                     }
                     if (bk.cur)                           // causal mask on the diagonal block
                         gs += pds_half<true>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, r_in, nullptr, ds_tile, row);
@@ -388,24 +428,25 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                         gs += pds_half<false>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, 63, nullptr, ds_tile, row);
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&bars->ds_full[t]);
+                mbar_arrive(&bars->ds_full[u]);
                 if (!bk.cur && bk.valid) {
                     gs = warp_sum(gs);
                     if (lane == 0) atomicAdd(p.gsum + it.row * p.K + k, gs * p.inv_scale);
                 }
             }
             if (!ok) break;
-            if (!mbar_wait(&bars->dq_full[t], q_it & 1, abort, p.status)) break;
-            ++q_it;
+            kb += it.nb;
+            // dQ of the item: warpgroup u writes dims [64 u, 64 u + 64) of its rows
+            if (!(ok = mbar_wait(&bars->dq_full, qn & 1, abort, p.status))) break;
             tc_fence_after();
             const long long orow = ((long long)it.b * p.S + (long long)it.i * 64 + r_in) * p.Hq + hq;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q2 = 0; q2 < 2; ++q2) {
                 uint32_t ov[32];
-                tmem_ld32(tQ + q4 * 32, ov);
+                tmem_ld32(tmem + lane_base + kTmDQ + 64 * u + 32 * q2, ov);
                 tmem_wait_ld();
                 if (row_ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.dq + orow * kD + q4 * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(p.dq + orow * kD + 64 * u + 32 * q2);
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
                         uint4 w;
@@ -418,7 +459,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->dq_empty[t]);
+            mbar_arrive(&bars->dq_empty);
         }
     }
     tc_fence_before();
@@ -860,7 +901,6 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     p.G = G;
     p.K = a.K;
     p.NQB = NQB;
-    p.ntg = ((G + 1) / 2 + 1) / 2;
     p.ntile = (G + 1) / 2;
     p.idx = a.idx;
     p.cnt = a.cnt;
@@ -881,11 +921,11 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
-    p.n_items = a.B * a.Hkv * NQB * p.ntg;
+    p.n_items = a.B * a.Hkv * NQB * p.ntile;
     if ((e = cudaFuncSetAttribute(dqk::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dqk::kSmem)) !=
         cudaSuccess)
         return e;
-    dqk::dq_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, dqk::kSmem, st>>>(mq, mdo, mk, mv, p);
+    dqk::dq_kernel<<<p.n_items < sms ? p.n_items : sms, dqk::kThreadsDq, dqk::kSmem, st>>>(mq, mdo, mk, mv, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     p.n_items = a.B * a.Hkv * NQB;

@@ -18,8 +18,9 @@
 //    gradients (warp sums of dS).
 //  * dkv_kernel (key-stationary): item = (b, h, j); walks the query blocks
 //    that attend block j (its own block and every block that kept it, from a
-//    reverse index), one Q tile per step, and accumulates dV^T = sum dO^T P
-//    and dK^T = sum Q^T dS in TMEM (M = head dim).
+//    reverse index), one Q tile per step streamed through a 5-slot ring,
+//    and accumulates dV^T = sum dO^T P and dK^T = sum Q^T dS in TMEM
+//    (M = head dim); both softmax warpgroups work on every step.
 // S and dP are computed twice (once per kernel) instead of once; in exchange
 // nothing is reduced through global memory and dq/dk/dv are deterministic.
 //
@@ -475,19 +476,28 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
 // ==================================================================== dk, dv
 namespace dkv {
 
+// K_j, V_j stay in shared memory for the item; the steps' Q and dO tiles
+// (32 KiB each) stream through a ring of five slots, Q of step g in slot
+// 2g mod 5 and dO in slot 2g+1 mod 5, so two and a half steps are in flight.
 constexpr uint32_t kOffK = 0;                      // K_j: 64 keys x 256 B
 constexpr uint32_t kOffV = kBlk;                   // V_j
-constexpr uint32_t kOffStage = 2 * kBlk;           // 2 stages x (Q tile, dO tile)
-constexpr int kNS = 2;
-constexpr uint32_t kStage = 2 * kTile;
-constexpr uint32_t kOffPS = kOffStage + kNS * kStage;    // per warpgroup: P tile, dS tile
-constexpr uint32_t kOffBar = kOffPS + 2 * 2 * kRowTile;  // 224 KB
+constexpr uint32_t kOffRing = 2 * kBlk;
+constexpr int kSlots = 5;
+constexpr uint32_t kOffP = kOffRing + kSlots * kTile;    // P tile, then dS tile of the current step
+constexpr uint32_t kOffDS = kOffP + kRowTile;
+constexpr uint32_t kOffBar = kOffDS + kRowTile;          // 224 KB
 constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
+// TMEM columns: S/dP buffer b (steps of parity b) at 128 b (S, dP + 64); dV^T, dK^T accumulators
+constexpr uint32_t kTmAccV = 256, kTmAccK = 320;
+
+// warps: 0 TMA; 2-5 / 6-9 softmax warpgroups 0 / 1 (both on every step, keys
+// [32 w, 32 w + 32)); issuing warps 1: S = Q K^T, 10: dP = dO V^T,
+// 11: dV^T += dO^T P, 12: dK^T += Q^T dS
 
 struct Bars {
     uint64_t kv_full, kv_empty;
-    uint64_t qd_full[kNS], qd_empty[kNS];
-    uint64_t s_full[2], tm_free[2], pds_full[2], pds_empty[2];
+    uint64_t q_full[kSlots], o_full[kSlots], slot_empty[kSlots];
+    uint64_t s_full[2], tm_free[2], pds_full, pds_empty;
     uint64_t acc_full, acc_empty;
     uint64_t drain[4];
     uint32_t tmem_base;
@@ -548,20 +558,21 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     volatile int* abort = &bars->abort;
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
-        mbar_init(&bars->kv_empty, 4);                  // one arrival per issuing warp
-        for (int s = 0; s < kNS; ++s) {
-            mbar_init(&bars->qd_full[s], 1);
-            mbar_init(&bars->qd_empty[s], 2);           // the two warps of the step's warpgroup
+        mbar_init(&bars->kv_empty, 2);                  // the S and dP warps
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->o_full[s], 1);
+            mbar_init(&bars->slot_empty[s], 1);         // the tile's last reader (dK^T or dV^T warp)
         }
-        for (int w = 0; w < 2; ++w) {
-            mbar_init(&bars->s_full[w], 2);
-            mbar_init(&bars->tm_free[w], 128);
-            mbar_init(&bars->pds_full[w], 128);
-            mbar_init(&bars->pds_empty[w], 2);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->s_full[b], 2);
+            mbar_init(&bars->tm_free[b], 256);
         }
-        for (int w = 0; w < 4; ++w) mbar_init(&bars->drain[w], 1);
-        mbar_init(&bars->acc_full, 4);
+        mbar_init(&bars->pds_full, 256);
+        mbar_init(&bars->pds_empty, 2);
+        mbar_init(&bars->acc_full, 2);
         mbar_init(&bars->acc_empty, 256);
+        for (int w = 0; w < 4; ++w) mbar_init(&bars->drain[w], 1);
         bars->abort = 0;
         fence_barrier_init();
     }
@@ -576,9 +587,9 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     const uint32_t s_base = smem_u32(smem);
 
     if (warp == 0) {
+        // ---------------------------------------------------------------- TMA
         if (lane == 0) {
-            uint32_t item_it = 0, qd_it = 0;
-            int last_it[kNS] = {-1, -1};
+            uint32_t item_it = 0, g = 0, npos = 0;      // npos: Q / dO tiles issued
             bool kv_issued = false;
             for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x, ++item_it) {
                 int b, h, j;
@@ -593,113 +604,127 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 }
                 kv_issued = true;
                 const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
-                for (int e = 0; e < n && !*abort; ++e) {
+                bool ok = true;
+                for (int e = 0; e < n && ok; ++e) {
                     int i = __ldg(list + e) >> 16;
                     if (i < j || i >= p.NQB) {
                         flag_status(p.status, kStatusBadData);
                         i = j;
                     }
-                    for (int t = 0; t < p.ntile; ++t, ++qd_it) {
-                        const int st = qd_it % kNS;
-                        if (!mbar_wait(&bars->qd_empty[st], ((qd_it / kNS) & 1) ^ 1, abort, p.status)) break;
-                        mbar_expect_tx(&bars->qd_full[st], 8 * kBox);
-                        for (int s = 0; s < 2; ++s) {
-                            const int slot = 2 * t + s;
-                            const int hq = h * p.G + (slot < p.G ? slot : 0);
-                            for (int a = 0; a < 2; ++a) {
-                                const uint32_t off = kOffStage + st * kStage + a * kTileAtom + s * kBox;
-                                tma_load_3d(smem + off, &map_q, &bars->qd_full[st], a * 64, hq, b * p.S + i * 64);
-                                tma_load_3d(smem + off + kTile, &map_do, &bars->qd_full[st], a * 64, hq,
-                                            b * p.S + i * 64);
+                    for (int t = 0; t < p.ntile && ok; ++t, ++g) {
+                        // Q of step g, then its dO, each into the next ring slot
+                        for (int part = 0; part < 2 && ok; ++part) {
+                            const uint32_t pos = 2 * g + part;
+                            const int sl = pos % kSlots;
+                            if (!(ok = mbar_wait(&bars->slot_empty[sl], ((pos / kSlots) & 1) ^ 1, abort, p.status))) break;
+                            uint64_t* fb = part == 0 ? &bars->q_full[sl] : &bars->o_full[sl];
+                            const CUtensorMap* mp = part == 0 ? &map_q : &map_do;
+                            mbar_expect_tx(fb, 4 * kBox);
+                            for (int s = 0; s < 2; ++s) {
+                                const int hs = 2 * t + s;
+                                const int hq = h * p.G + (hs < p.G ? hs : 0);
+                                for (int a = 0; a < 2; ++a)
+                                    tma_load_3d(smem + kOffRing + sl * kTile + a * kTileAtom + s * kBox, mp, fb, a * 64,
+                                                hq, b * p.S + i * 64);
                             }
+                            ++npos;
                         }
-                        last_it[st] = (int)qd_it;
                     }
                 }
+                if (!ok) break;
             }
-            if (*abort) {
+            if (*abort) {           // let every copy in flight land before the CTA exits
                 volatile int no_abort = 0;
-                for (int s = 0; s < kNS; ++s)
-                    if (last_it[s] >= 0)
-                        mbar_wait(&bars->qd_full[s], ((uint32_t)last_it[s] / kNS) & 1, &no_abort, nullptr);
+                for (uint32_t pos = npos > (uint32_t)kSlots ? npos - kSlots : 0u; pos < npos; ++pos) {
+                    const uint32_t gg = pos / 2;
+                    mbar_wait(pos & 1 ? &bars->o_full[pos % kSlots] : &bars->q_full[pos % kSlots], (gg / kSlots) & 1,
+                              &no_abort, nullptr);
+                }
                 if (kv_issued) mbar_wait(&bars->kv_full, (item_it - 1) & 1, &no_abort, nullptr);
             }
         }
     } else if (is_issuer_warp(warp)) {
-        // Step m of an item belongs to warpgroup w = m % 2. For warpgroup w, slot w
-        // issues S = Q K^T and dK^T += Q^T dS, slot 2 + w issues dP = dO V^T and
-        // dV^T += dO^T P, each into its own accumulator (the drain adds the two
-        // warpgroups' halves). The whole warp runs the loop, one lane issues.
-        const int slot = issuer_slot(warp);
-        const int w = slot & 1;
-        const bool xq = slot < 2;                       // the Q side (else the dO side)
-        const uint32_t id_s = idesc_bf16(128, 64, false, false);
-        const uint32_t id_t = idesc_bf16(128, 64, true, true);
-        const uint32_t kv_lo = sdesc_lo(s_base + (xq ? kOffK : kOffV), 16);
-        const uint32_t a_off = xq ? 0u : kTile;         // Q or dO inside a stage
-        const uint32_t d_sp = tmem + 128 * w + (xq ? 0u : 64u);
-        // accumulator: dV^T of warpgroup w at 256 + 128 w, dK^T at + 64
-        const uint32_t acc = tmem + 256 + 128 * w + (xq ? 64u : 0u);
-        // B of the accumulation: P (dO side) or dS (Q side) of warpgroup w, MN-major
-        const uint32_t pb_lo = sdesc_lo(s_base + kOffPS + w * 2 * kRowTile + (xq ? kRowTile : 0u), kRowTile);
-        uint32_t item_it = 0, gbase = 0, pds_it = 0, sdp_n = 0;
+        // ----------------------------------------------------- issuing warps
+        const int slot = issuer_slot(warp);             // 0: S, 1: dP, 2: dV^T, 3: dK^T
+        uint32_t item_it = 0, g = 0;
         bool ok = true;
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
-            int b, h, j;
-            long long bh;
-            item_of(p, id, b, h, j, bh);
-            const int N = n_entries(p, bh, j) * p.ntile;
-            if (!(ok = mbar_wait_warp(&bars->kv_full, item_it & 1, abort, p.status))) break;
-            // the drain of the previous item has read both accumulators
-            if (!(ok = mbar_wait_warp(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
-            tc_fence_after();
-            for (int m = w; m < N && ok; m += 2) {
-                const uint32_t g = gbase + m;
-                const int st = g % kNS;
-                if (!(ok = mbar_wait_warp(&bars->qd_full[st], (g / kNS) & 1, abort, p.status))) break;
-                // this warpgroup has loaded its previous S/dP out of TMEM
-                if (sdp_n > 0 && !(ok = mbar_wait_warp(&bars->tm_free[w], (sdp_n - 1) & 1, abort, p.status))) break;
-                ++sdp_n;
-                tc_fence_after();
-                const uint32_t a_lo = sdesc_lo(s_base + kOffStage + st * kStage + a_off, 16);   // K-major Q / dO
+        if (slot < 2) {
+            const bool is_s = slot == 0;
+            const uint32_t id_s = idesc_bf16(128, 64, false, false);
+            const uint32_t kv_lo = sdesc_lo(s_base + (is_s ? kOffK : kOffV), 16);
+            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+                int b, h, j;
+                long long bh;
+                item_of(p, id, b, h, j, bh);
+                const int N = n_entries(p, bh, j) * p.ntile;
+                if (!(ok = mbar_wait_warp(&bars->kv_full, item_it & 1, abort, p.status))) break;
+                for (int m = 0; m < N && ok; ++m, ++g) {
+                    const uint32_t pos = 2 * g + (is_s ? 0 : 1);
+                    const int sl = pos % kSlots;
+                    if (!(ok = mbar_wait_warp(is_s ? &bars->q_full[sl] : &bars->o_full[sl], (g / kSlots) & 1, abort,
+                                              p.status)))
+                        break;
+                    // both warpgroups have read the previous S / dP of this buffer out of TMEM
+                    const int buf = g & 1;
+                    if (g >= 2 && !(ok = mbar_wait_warp(&bars->tm_free[buf], ((g - 2) >> 1) & 1, abort, p.status)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t a_lo = sdesc_lo(s_base + kOffRing + sl * kTile, 16);   // K-major Q / dO
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
-                    mma_ss_e(d_sp, a_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi, id_s, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ao = (kk >> 2) * kTileAtom + (kk & 3) * 32;
+                        const uint32_t bo = (kk >> 2) * kBlkAtom + (kk & 3) * 32;
+                        mma_ss_e(tmem + 128 * buf + (is_s ? 0u : 64u), a_lo + (ao >> 4), kHi, kv_lo + (bo >> 4), kHi,
+                                 id_s, kk > 0);
+                    }
+                    mma_commit_e(&bars->s_full[buf]);
                 }
-                mma_commit_e(&bars->s_full[w]);
-                // the accumulation once the warpgroup wrote P and dS
-                if (!(ok = mbar_wait_warp(&bars->pds_full[w], pds_it & 1, abort, p.status))) break;
-                ++pds_it;
-                tc_fence_after();
-                const uint32_t at_lo = sdesc_lo(s_base + kOffStage + st * kStage + a_off, kTileAtom);   // MN-major
-                const uint32_t acc0 = (m >= 2) ? 1u : 0u;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_e(acc, at_lo + ((kk * 2048) >> 4), kHi, pb_lo + ((kk * 2048) >> 4), kHi, id_t,
-                             kk > 0 ? 1u : acc0);
-                mma_commit_e(&bars->qd_empty[st]);
-                mma_commit_e(&bars->pds_empty[w]);
+                if (!ok) break;
+                mma_commit_e(&bars->kv_empty);          // K_j / V_j may be replaced
             }
-            if (!ok) break;
-            gbase += N;
-            mma_commit_e(&bars->kv_empty);
-            mma_commit_e(&bars->acc_full);
+        } else {
+            // dV^T += dO^T P (slot 2) or dK^T += Q^T dS (slot 3): A = the step's dO / Q
+            // tile MN-major, B = P / dS MN-major
+            const bool is_v = slot == 2;
+            const uint32_t id_t = idesc_bf16(128, 64, true, true);
+            const uint32_t acc = tmem + (is_v ? kTmAccV : kTmAccK);
+            const uint32_t pb_lo = sdesc_lo(s_base + (is_v ? kOffP : kOffDS), kRowTile);
+            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+                int b, h, j;
+                long long bh;
+                item_of(p, id, b, h, j, bh);
+                const int N = n_entries(p, bh, j) * p.ntile;
+                // the drain of the previous item has read the accumulators
+                if (!(ok = mbar_wait_warp(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
+                for (int m = 0; m < N && ok; ++m, ++g) {
+                    if (!(ok = mbar_wait_warp(&bars->pds_full, g & 1, abort, p.status))) break;
+                    tc_fence_after();
+                    const int sl = (2 * g + (is_v ? 1 : 0)) % kSlots;
+                    const uint32_t at_lo = sdesc_lo(s_base + kOffRing + sl * kTile, kTileAtom);   // MN-major
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss_e(acc, at_lo + ((kk * 2048) >> 4), kHi, pb_lo + ((kk * 2048) >> 4), kHi, id_t,
+                                 (m > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit_e(&bars->slot_empty[sl]);   // the tile's last reader
+                    mma_commit_e(&bars->pds_empty);
+                }
+                if (!ok) break;
+                mma_commit_e(&bars->acc_full);
+            }
         }
         mma_commit_e(&bars->drain[slot]);
         volatile int no_abort = 0;
         mbar_wait(&bars->drain[slot], 0, &no_abort, nullptr);
-    } else if (warp >= 2 && warp < 10) {
-        const int w = (warp - 2) >> 2;
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        const int w = (warp - 2) >> 2;                  // keys [32 w, 32 w + 32) of every step
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int r_in = row & 63;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_base + 128 * w;
-        uint8_t* bufP = smem + kOffPS + w * 2 * kRowTile;
-        uint8_t* bufS = bufP + kRowTile;
-        uint32_t s_it = 0, pds_n = 0, item_it = 0;
+        uint8_t* bufP = smem + kOffP;
+        uint8_t* bufS = smem + kOffDS;
+        uint32_t item_it = 0, g = 0;
         bool ok = true;
         for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
             int b, h, j;
@@ -707,46 +732,38 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             item_of(p, id, b, h, j, bh);
             const int N = n_entries(p, bh, j) * p.ntile;
             const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
-            // metadata pipeline: entry of step m + 4 and loads of step m + 2 in flight
-            int ent2 = (w + 2 < N) ? __ldg(list + (w + 2) / p.ntile) : 0;
-            StepMeta nxt;
-            if (w < N) nxt = step_meta(p, __ldg(list + w / p.ntile), b, h, bh, j, w, row);
-            for (int m = w; m < N; m += 2) {
+            // metadata pipeline: entry of step m + 2 and loads of step m + 1 in flight
+            int ent2 = (1 < N) ? __ldg(list + 1 / p.ntile) : 0;
+            StepMeta nxt = step_meta(p, __ldg(list), b, h, bh, j, 0, row);
+            for (int m = 0; m < N; ++m, ++g) {
                 const StepMeta sm = nxt;
-                if (m + 2 < N) nxt = step_meta(p, ent2, b, h, bh, j, m + 2, row);
-                if (m + 4 < N) ent2 = __ldg(list + (m + 4) / p.ntile);
-                if (!(ok = mbar_wait(&bars->s_full[w], s_it & 1, abort, p.status))) break;
-                ++s_it;
+                if (m + 1 < N) nxt = step_meta(p, ent2, b, h, bh, j, m + 1, row);
+                if (m + 2 < N) ent2 = __ldg(list + (m + 2) / p.ntile);
+                const int buf = g & 1;
+                if (!(ok = mbar_wait(&bars->s_full[buf], (g >> 1) & 1, abort, p.status))) break;
                 tc_fence_after();
                 const bool valid = sm.in_range && (sm.cur || (sm.slot < p.K && sm.idxv == j));
                 // log2 domain; rows of an absent head (or a bad entry) get -inf: P = dS = 0
                 const float off = (valid && sm.row_ok) ? sm.lg * kLog2e - sm.lse * kLog2e : -INFINITY;
                 const float drs = sm.drow * p.sm_scale;
-                // the MMA of this warpgroup's previous step has finished reading the buffers
-                if (pds_n > 0 && !(ok = mbar_wait(&bars->pds_empty[w], (pds_n - 1) & 1, abort, p.status))) break;
-                ++pds_n;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {          // keys [32 hf, 32 hf + 32)
-                    uint32_t sv[32], pv[32];
-                    tmem_ld32(tS + 32 * hf, sv);
-                    tmem_ld32(tS + 64 + 32 * hf, pv);
-                    tmem_wait_ld();
-                    if (hf == 1) {
-                        tc_fence_before();
-                        mbar_arrive(&bars->tm_free[w]);   // S/dP columns may be refilled
-                    }
-                    if (sm.cur)                           // causal mask on the diagonal block
-                        pds_half<true>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, r_in, bufP, bufS, row);
-                    else
-                        pds_half<false>(sv, pv, hf, p.scale2, off, p.sm_scale, drs, 63, bufP, bufS, row);
-                }
+                uint32_t sv[32], pv[32];
+                const uint32_t tS = tmem + lane_base + 128 * buf + 32 * w;
+                tmem_ld32(tS, sv);
+                tmem_ld32(tS + 64, pv);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&bars->tm_free[buf]);       // S/dP columns may be refilled
+                // the accumulation MMAs of the previous step have read the P / dS tiles
+                if (g > 0 && !(ok = mbar_wait(&bars->pds_empty, (g - 1) & 1, abort, p.status))) break;
+                if (sm.cur)                             // causal mask on the diagonal block
+                    pds_half<true>(sv, pv, w, p.scale2, off, p.sm_scale, drs, r_in, bufP, bufS, row);
+                else
+                    pds_half<false>(sv, pv, w, p.scale2, off, p.sm_scale, drs, 63, bufP, bufS, row);
                 fence_proxy_async_smem();
-                mbar_arrive(&bars->pds_full[w]);
+                mbar_arrive(&bars->pds_full);
             }
             if (!ok) break;
-            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim
-            // index); each is the sum of the two issuers' accumulators (issuer 1
-            // has none when the item has a single step)
+            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim index)
             if (!(ok = mbar_wait(&bars->acc_full, item_it & 1, abort, p.status))) break;
             tc_fence_after();
             {
@@ -754,18 +771,14 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 __nv_bfloat16* out = (w == 0 ? p.dv : p.dk) + ((long long)b * p.S + (long long)j * 64) * p.Hkv * kD +
                                      (long long)h * kD + d;
                 const long long key_stride = (long long)p.Hkv * kD;
-                const bool two = N > 1;
 #pragma unroll 1
                 for (int qt = 0; qt < 4; ++qt) {
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16(tmem + lane_base + 256 + 64 * w + 16 * qt, v0);
-                    tmem_ld16(tmem + lane_base + 384 + 64 * w + 16 * qt, v1);
+                    uint32_t v0[16];
+                    tmem_ld16(tmem + lane_base + (w == 0 ? kTmAccV : kTmAccK) + 16 * qt, v0);
                     tmem_wait_ld();
                     __nv_bfloat16* o2 = out + 16 * qt * key_stride;
 #pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        o2[u * key_stride] =
-                            __float2bfloat16_rn(__uint_as_float(v0[u]) + (two ? __uint_as_float(v1[u]) : 0.f));
+                    for (int u = 0; u < 16; ++u) o2[u * key_stride] = __float2bfloat16_rn(__uint_as_float(v0[u]));
                 }
             }
             tc_fence_before();

@@ -2,15 +2,18 @@
 
     python -m trainable_gated_block_b200.run_once --workload qwen3-4b-8k --reps 2
     python -m trainable_gated_block_b200.run_once --workload decode-64seq --reps 2
+    python -m trainable_gated_block_b200.run_once --workload decode-64seq --seqs 16 --reps 1
 
 A prefill workload runs select -> forward -> backward; a decode workload runs
 select -> paged decode. Nothing is timed or checked here: this is the command
 that ncu captures wrap (the numbers come from bench.py and the checks from
-the tests).
+the tests). ``--seqs`` keeps the first sequences of a decode workload only,
+so that a full capture holds a few GB on the device.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import math
 
 import torch
@@ -22,9 +25,12 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="qwen3-4b-8k")
     ap.add_argument("--reps", type=int, default=2)
+    ap.add_argument("--seqs", type=int, default=0, help="decode: use this many sequences")
     a = ap.parse_args()
     build.build()
     cfg = inputs.workload(a.workload)
+    if a.seqs and isinstance(cfg, inputs.DecodeConfig):
+        cfg = dataclasses.replace(cfg, N=a.seqs)
     if isinstance(cfg, inputs.DecodeConfig):
         x = {k: v.cuda() for k, v in inputs.make_decode(cfg).items()}
         ws = torch.empty(sas.decode_workspace_bytes(cfg.N, cfg.Hq, cfg.Hkv, cfg.D, cfg.K), dtype=torch.uint8,

@@ -796,22 +796,44 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 }  // namespace dkv
 
 // ================================================================ helpers
-__global__ void dot_rows_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                                long long rows, int S, int Hq, float* __restrict__ Dr) {
-    // one warp per (b, t, hq) row of 128; Dr as [B, Hq, S]
-    const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (w >= rows) return;
-    const uint2 a = reinterpret_cast<const uint2*>(o + w * kD)[lane];
-    const uint2 c = reinterpret_cast<const uint2*>(dout + w * kD)[lane];
-    float2 a0 = bf16x2_to_f32(a.x), a1 = bf16x2_to_f32(a.y), c0 = bf16x2_to_f32(c.x), c1 = bf16x2_to_f32(c.y);
-    float acc = a0.x * c0.x + a0.y * c0.y + a1.x * c1.x + a1.y * c1.y;
-    acc = warp_sum(acc);
-    if (lane == 0) {
-        const int hq = (int)(w % Hq);
-        const long long bt = w / Hq;
-        const long long b = bt / S, t = bt % S;
-        Dr[(b * Hq + hq) * S + t] = acc;
+// Dr = rowsum(O * dO) over D = 128 for every (b, t, hq) row; Dr as [B, Hq, S].
+// HBM-bound: a warp takes 8 consecutive rows, 16 lanes per row with 16-byte
+// loads, all eight loads of a lane issued before any is used.
+constexpr int kDotRowsPerWarp = 8;
+__global__ void __launch_bounds__(256) dot_rows_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout, long long rows, int S,
+                                                       int Hq, float* __restrict__ Dr) {
+    const long long w0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kDotRowsPerWarp;
+    const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
+    uint4 a[kDotRowsPerWarp / 2], c[kDotRowsPerWarp / 2];
+#pragma unroll
+    for (int r = 0; r < kDotRowsPerWarp / 2; ++r) {
+        const long long row = w0 + 2 * r + half;
+        a[r] = c[r] = make_uint4(0u, 0u, 0u, 0u);
+        if (row < rows) {
+            a[r] = __ldg(reinterpret_cast<const uint4*>(o + row * kD) + l16);
+            c[r] = __ldg(reinterpret_cast<const uint4*>(dout + row * kD) + l16);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kDotRowsPerWarp / 2; ++r) {
+        const uint32_t* x = reinterpret_cast<const uint32_t*>(&a[r]);
+        const uint32_t* y = reinterpret_cast<const uint32_t*>(&c[r]);
+        float acc = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = bf16x2_to_f32(x[q]), g = bf16x2_to_f32(y[q]);
+            acc = fmaf(f.x, g.x, fmaf(f.y, g.y, acc));
+        }
+#pragma unroll
+        for (int m = 8; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        const long long row = w0 + 2 * r + half;
+        if (l16 == 0 && row < rows) {
+            const int hq = (int)(row % Hq);
+            const long long bt = row / Hq;
+            const long long b = bt / S, t = bt % S;
+            Dr[(b * Hq + hq) * S + t] = acc;
+        }
     }
 }
 
@@ -899,8 +921,9 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     if ((e = cudaMemsetAsync(ws.gsum, 0, sizeof(float) * (size_t)bhq * (a.K > 0 ? a.K : 1), st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(ws.slotmap, 0, sizeof(int16_t) * (size_t)bhq * NQB, st)) != cudaSuccess) return e;
     const long long drows = rows * a.Hq;
-    dot_rows_kernel<<<(unsigned)((drows + 7) / 8), 256, 0, st>>>((const __nv_bfloat16*)bw.o,
-                                                                 (const __nv_bfloat16*)bw.dout, drows, a.S, a.Hq, ws.Dr);
+    const long long dwarps = (drows + kDotRowsPerWarp - 1) / kDotRowsPerWarp;
+    dot_rows_kernel<<<(unsigned)((dwarps + 7) / 8), 256, 0, st>>>((const __nv_bfloat16*)bw.o,
+                                                                  (const __nv_bfloat16*)bw.dout, drows, a.S, a.Hq, ws.Dr);
     rev_fill_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(a.idx, a.cnt, bhq, NQB, a.K, ws.slotmap);
     rev_list_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(ws.slotmap, bhq, NQB, ws.rlist, ws.rcount);
     count_launches(3);

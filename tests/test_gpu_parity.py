@@ -76,15 +76,16 @@ def test_select_full_workloads(name):
     _select_checks(s, cfg.K, gsel, O.prefill_history(NQB))
 
 
-def test_select_adversarial_ties():
+@pytest.mark.parametrize("R", [200, 700])     # one-warp rows, and one-CTA rows (> 512 history)
+def test_select_adversarial_ties(R):
     rng = np.random.default_rng(5)
-    B, H, R = 2, 3, 200
+    B, H = 2, 3
     s = rng.choice(np.array([-1.0, -0.0, 0.0, 0.5, 2.0], dtype=np.float32), size=(B, H, R, R))
     s[0, 0] = 0.25                        # all-equal rows
     s[0, 1, :, ::2] = -0.0                # +/- zero ties
     s[0, 1, :, 1::2] = 0.0
     st = torch.from_numpy(s)
-    for K in (0, 1, 7, 32, 199, 300):
+    for K in (0, 1, 7, 32, 199, 300, R + 5):
         gsel = sas.select(_poisoned(st).cuda(), K)
         sas.get_error_flag()
         _select_checks(st, K, gsel, O.prefill_history(R))

@@ -363,34 +363,35 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
         uint8_t* ds_tile = smem + kOffDS + u * kRowTile;
         uint32_t kb = 0, qn = 0, s_it = 0, ds_n = 0;
         bool ok = true;
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
-            const Item it = item_of(p, id);
-            // copy this warpgroup's half of the staged tile (0: Q, 1: dO) into TMEM once
-            // the S / dP warps are done with the previous item's
-            if (qn > 0 && !(ok = mbar_wait(&bars->qt_free, (qn - 1) & 1, abort, p.status))) break;
-            if (!(ok = mbar_wait(&bars->qs_full, qn & 1, abort, p.status))) break;
-            {
-                const uint8_t* src = smem + kOffQs + u * kTile;
-                const uint32_t dst = tmem + lane_base + (u == 0 ? kTmQ : kTmO);
+        // copy this warpgroup's half of staged tile number n (0: Q, 1: dO) into TMEM
+        // once the S / dP warps are done with the previous item's
+        auto copy_qd = [&](uint32_t n) -> bool {
+            if (n > 0 && !mbar_wait(&bars->qt_free, (n - 1) & 1, abort, p.status)) return false;
+            if (!mbar_wait(&bars->qs_full, n & 1, abort, p.status)) return false;
+            const uint8_t* src = smem + kOffQs + u * kTile;
+            const uint32_t dst = tmem + lane_base + (u == 0 ? kTmQ : kTmO);
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {           // dims [64 a, 64 a + 64) -> 32 packed columns
-                    uint32_t v[32];
+            for (int a = 0; a < 2; ++a) {               // dims [64 a, 64 a + 64) -> 32 packed columns
+                uint32_t v[32];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(src + a * kTileAtom + sw128_offset(row, c));
-                        v[4 * c] = w.x;
-                        v[4 * c + 1] = w.y;
-                        v[4 * c + 2] = w.z;
-                        v[4 * c + 3] = w.w;
-                    }
-                    tmem_st32(dst + 32 * a, v);
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(src + a * kTileAtom + sw128_offset(row, c));
+                    v[4 * c] = w.x;
+                    v[4 * c + 1] = w.y;
+                    v[4 * c + 2] = w.z;
+                    v[4 * c + 3] = w.w;
                 }
-                tmem_wait_st();
+                tmem_st32(dst + 32 * a, v);
             }
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->qs_empty);
             mbar_arrive(&bars->qt_full);
-
+            return true;
+        };
+        if (blockIdx.x < p.n_items) ok = copy_qd(0);
+        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
+            const Item it = item_of(p, id);
             const int slot = 2 * it.t + slot_in_tile;
             const bool row_ok = slot < p.G;
             const int hq = it.h * p.G + (row_ok ? slot : 0);
@@ -437,6 +438,9 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             }
             if (!ok) break;
             kb += it.nb;
+            // the next item's Q / dO go into TMEM first, so that its S / dP start
+            // while this item's dQ is written out
+            if (id + (int)gridDim.x < p.n_items && !(ok = copy_qd(qn + 1))) break;
             // dQ of the item: warpgroup u writes dims [64 u, 64 u + 64) of its rows
             if (!(ok = mbar_wait(&bars->dq_full, qn & 1, abort, p.status))) break;
             tc_fence_after();

@@ -23,7 +23,9 @@
 //               (one TMEM lane); logits = sm_scale q.k + log-gate in the log2
 //               domain, causal mask on the diagonal block, running max/sum;
 //               P (bf16) over the consumed S buffer; O in TMEM rescaled only
-//               when the max grows by more than 2^8; final o and row LSE.
+//               when the max grows by more than 2^8 (the only point, besides
+//               the end of the item, where the softmax waits for a PV: the
+//               issuer publishes completed PVs as a count); final o and LSE.
 // TMEM (512 columns): tile t owns [256t, 256t+256): S buffers at +0 and +64
 // (64 columns each, P overwrites the first 32), O at +128.
 #include "launch.h"
@@ -65,7 +67,29 @@ struct Bars {
     uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
+    uint32_t pv_count[2];    // PVs of tile t known complete (issuer writes, softmax polls)
 };
+
+// Bounded wait until the published count reaches `target` (acquire); gives up
+// like mbar_wait: on the abort flag or after about kWaitCycles clocks.
+__device__ __forceinline__ bool wait_count(const uint32_t* c, uint32_t target, volatile int* abort, int* status) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(c)) : "memory");
+    if ((int)(v - target) >= 0) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(c)) : "memory");
+        if ((int)(v - target) >= 0) return true;
+        if ((it & 63u) == 0) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitCycles) {
+                *abort = 1;
+                flag_status(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
 
 struct Params {
     int B, S, Hq, Hkv, G, K, NQB, ntg, n_items;
@@ -147,6 +171,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         mbar_init(&bars->drain[0], 1);
         mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
+        bars->pv_count[0] = bars->pv_count[1] = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -220,7 +245,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int t = (warp == 1) ? 0 : 1;
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_pv = idesc_bf16(128, kD, false, true);
-            uint32_t kv_it = 0, q_it = 0, p_it[2] = {0, 0}, oe_it = 0;
+            uint32_t kv_it = 0, q_it = 0, p_it[2] = {0, 0}, oe_it = 0, pv_n = 0;
             constexpr uint32_t kHi = sdesc_hi(1024);
             const uint32_t q_lo = sdesc_lo(sQ + t * kQTile, 16);
             auto issue_s = [&](int st, int buf) {
@@ -283,6 +308,12 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (k + 3 == it.nb)
                         for (int c = 0; c < owe; ++c) mma_commit(&bars->q_empty);
                     for (int c = 0; c < owe; ++c) mma_commit(&bars->kv_empty[st]);
+                    // publish PV completion: the softmax waits for it only when it
+                    // rescales O and at the end of the item
+                    if (!(ok = mbar_wait(&bars->o_done[t], pv_n & 1, abort, p.status))) break;
+                    ++pv_n;
+                    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_u32(&bars->pv_count[t])), "r"(pv_n)
+                                 : "memory");
                 }
             }
             mma_commit(&bars->drain[t]);
@@ -298,8 +329,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t tT = tmem + lane_base + 256 * t;
         const uint32_t tO = tT + 128;
-        // o_done[t] completes once per PV of this tile; it is waited on phase by
-        // phase (a parity wait is exact only within one phase of the barrier).
+        // pv_count[t]: PVs of this tile completed so far (published by the issuer)
         uint32_t s_it[2] = {0, 0}, pv_it = 0;
         for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
             const Item it = item_of(p, id);
@@ -337,12 +367,9 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
                 const float m_new = fmaxf(m_ref, mx);
                 const bool need = m_new > m_ref + kRescaleThreshold;
-                if (k > 0) {
-                    // PV of the previous step is done: O may be rescaled, and the
-                    // o_done phases are observed one by one
-                    if (!(ok = mbar_wait(&bars->o_done[t], (pv_it + k - 1) & 1, abort, p.status))) break;
-                }
                 if (__any_sync(0xffffffffu, need) && k > 0) {
+                    // O is rescaled in TMEM: PV of the previous step must be complete
+                    if (!(ok = wait_count(&bars->pv_count[t], pv_it + k, abort, p.status))) break;
                     tc_fence_after();
                     const float f = need ? exp2f(m_ref - m_new) : 1.f;
 #pragma unroll
@@ -374,7 +401,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 mbar_arrive(&bars->p_full[t][buf]);
             }
             if (!ok) break;
-            if (!mbar_wait(&bars->o_done[t], (pv_it + it.nb - 1) & 1, abort, p.status)) break;
+            if (!wait_count(&bars->pv_count[t], pv_it + it.nb, abort, p.status)) break;
             pv_it += it.nb;
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;

@@ -63,6 +63,7 @@ struct Params {
     const float* Dr;        // [B, Hq, S]
     const int32_t* rlist;   // [B, Hkv, NQB, NQB]: (i << 16) | slot, slot 0xFFFF = own block
     const int32_t* rcount;  // [B, Hkv, NQB]
+    const int32_t* order;   // dk/dv items sorted by decreasing step count
     float scale2;           // sm_scale * log2(e)
     float sm_scale;
     float inv_scale;        // 1 / sm_scale
@@ -84,7 +85,7 @@ template <bool kMask>
 __device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32_t (&pv)[32], int hf, float scale2,
                                           float off, float sm_scale, float drs, int lim, uint8_t* bufP,
                                           uint8_t* bufS, int row) {
-    float gs = 0.f;
+    float gs4[4] = {0.f, 0.f, 0.f, 0.f};          // 4 independent chains
 #pragma unroll
     for (int c = 0; c < 4; ++c) {                 // 16-byte chunk = keys 8c .. 8c+7 of the half
         uint32_t pp[4], dd[4];
@@ -98,7 +99,7 @@ __device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32
                 if (kMask) x = (32 * hf + e > lim) ? -INFINITY : x;
                 pr[q] = fast_exp2(x);
                 ds[q] = pr[q] * fmaf(__uint_as_float(pv[e]), sm_scale, -drs);
-                gs += ds[q];
+                gs4[e2] += ds[q];
             }
             pp[e2] = pack_bf16x2(pr[0], pr[1]);
             dd[e2] = pack_bf16x2(ds[0], ds[1]);
@@ -107,7 +108,7 @@ __device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32
         if (bufP) *reinterpret_cast<uint4*>(bufP + sw128_offset(row, ch)) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
         *reinterpret_cast<uint4*>(bufS + sw128_offset(row, ch)) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
     }
-    return gs;
+    return (gs4[0] + gs4[1]) + (gs4[2] + gs4[3]);
 }
 
 // ===================================================================== dq
@@ -521,6 +522,17 @@ __device__ __forceinline__ int n_entries(const Params& p, long long bh, int j) {
     return max(1, min(n, p.NQB - j));
 }
 
+// Item of this CTA's round r, or -1 past the end: the items sorted by
+// decreasing step count (dkv_order_kernel) are dealt to the CTAs in snake
+// order (forward on even rounds, backward on odd ones), so every CTA gets
+// about the same number of steps although a key block is attended by one to
+// hundreds of query blocks.
+__device__ __forceinline__ int item_at(const Params& p, int r) {
+    const int g = (int)gridDim.x;
+    const long long pos = (long long)r * g + ((r & 1) ? g - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return pos < p.n_items ? __ldg(p.order + pos) : -1;
+}
+
 // What a softmax thread needs for step m of item (b, h, j): the query block,
 // the gate of block j in that block's selection, and its row's LSE and Dr.
 // The reverse-list entry of a step is loaded two steps ahead and the loads
@@ -595,7 +607,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         if (lane == 0) {
             uint32_t item_it = 0, g = 0, npos = 0;      // npos: Q / dO tiles issued
             bool kv_issued = false;
-            for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x, ++item_it) {
+            for (int r = 0, id; (id = item_at(p, r)) >= 0 && !*abort; ++r, ++item_it) {
                 int b, h, j;
                 long long bh;
                 item_of(p, id, b, h, j, bh);
@@ -656,7 +668,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             const bool is_s = slot == 0;
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t kv_lo = sdesc_lo(s_base + (is_s ? kOffK : kOffV), 16);
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+            for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r, ++item_it) {
                 int b, h, j;
                 long long bh;
                 item_of(p, id, b, h, j, bh);
@@ -693,7 +705,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             const uint32_t id_t = idesc_bf16(128, 64, true, true);
             const uint32_t acc = tmem + (is_v ? kTmAccV : kTmAccK);
             const uint32_t pb_lo = sdesc_lo(s_base + (is_v ? kOffP : kOffDS), kRowTile);
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+            for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r, ++item_it) {
                 int b, h, j;
                 long long bh;
                 item_of(p, id, b, h, j, bh);
@@ -730,7 +742,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         uint8_t* bufS = smem + kOffDS;
         uint32_t item_it = 0, g = 0;
         bool ok = true;
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++item_it) {
+        for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r, ++item_it) {
             int b, h, j;
             long long bh;
             item_of(p, id, b, h, j, bh);
@@ -841,6 +853,39 @@ __global__ void __launch_bounds__(256) dot_rows_kernel(const __nv_bfloat16* __re
     }
 }
 
+// Sorts the dk/dv items (b, h, j) by decreasing step count (the length of
+// block j's reverse list) into `order`: 64 buckets of equal width, counted,
+// scanned by one warp and scattered; the order inside a bucket is arbitrary
+// (every item is computed on its own, so results do not depend on it).
+constexpr int kOrderBuckets = 64;
+__global__ void __launch_bounds__(1024) dkv_order_kernel(const int32_t* __restrict__ rcount, int n, int NQB,
+                                                         int32_t* __restrict__ order) {
+    __shared__ int cnt[kOrderBuckets], start[kOrderBuckets];
+    if (threadIdx.x < kOrderBuckets) cnt[threadIdx.x] = 0;
+    __syncthreads();
+    auto bucket = [&](int id) {
+        const int j = id % NQB;
+        const int c = max(1, min(rcount[id], NQB - j));      // steps of item id, 1..NQB
+        return (kOrderBuckets - 1) - (int)((long long)(c - 1) * kOrderBuckets / NQB);   // 0: largest
+    };
+    for (int id = threadIdx.x; id < n; id += blockDim.x) atomicAdd(&cnt[bucket(id)], 1);
+    __syncthreads();
+    if (threadIdx.x < 32) {                                   // exclusive scan over the buckets
+        const int l = threadIdx.x;
+        const int a = cnt[2 * l], b = cnt[2 * l + 1];
+        int s = a + b;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, s, d);
+            if (l >= d) s += t;
+        }
+        start[2 * l] = s - (a + b);
+        start[2 * l + 1] = s - b;
+    }
+    __syncthreads();
+    for (int id = threadIdx.x; id < n; id += blockDim.x) order[atomicAdd(&start[bucket(id)], 1)] = id;
+}
+
 __global__ void rev_fill_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int rows, int NQB,
                                 int K, int16_t* __restrict__ slotmap) {
     const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -883,6 +928,7 @@ struct Ws {
     int16_t* slotmap;
     int32_t* rlist;
     int32_t* rcount;
+    int32_t* order;
 };
 
 Ws carve(void* w, int B, int S, int Hq, int Hkv, int K) {
@@ -898,6 +944,8 @@ Ws carve(void* w, int B, int S, int Hq, int Hkv, int K) {
     r.rlist = reinterpret_cast<int32_t*>(p);
     p += align256(sizeof(int32_t) * (size_t)B * Hkv * NQB * NQB);
     r.rcount = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * (size_t)B * Hkv * NQB);
+    r.order = reinterpret_cast<int32_t*>(p);
     return r;
 }
 
@@ -908,7 +956,7 @@ size_t bwd_sm100_workspace(int B, int S, int Hq, int Hkv, int K) {
     return align256(sizeof(float) * (size_t)B * Hq * S) +
            align256(sizeof(float) * (size_t)B * Hkv * NQB * (size_t)(K > 0 ? K : 1)) +
            align256(sizeof(int16_t) * (size_t)B * Hkv * NQB * NQB) +
-           align256(sizeof(int32_t) * (size_t)B * Hkv * NQB * NQB) + align256(sizeof(int32_t) * (size_t)B * Hkv * NQB);
+           align256(sizeof(int32_t) * (size_t)B * Hkv * NQB * NQB) + 2 * align256(sizeof(int32_t) * (size_t)B * Hkv * NQB);
 }
 
 cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
@@ -930,7 +978,8 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
                                                                   (const __nv_bfloat16*)bw.dout, drows, a.S, a.Hq, ws.Dr);
     rev_fill_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(a.idx, a.cnt, bhq, NQB, a.K, ws.slotmap);
     rev_list_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(ws.slotmap, bhq, NQB, ws.rlist, ws.rcount);
-    count_launches(3);
+    dkv_order_kernel<<<1, 1024, 0, st>>>(ws.rcount, bhq, NQB, ws.order);
+    count_launches(4);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     Params p;
@@ -949,6 +998,7 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     p.Dr = ws.Dr;
     p.rlist = ws.rlist;
     p.rcount = ws.rcount;
+    p.order = ws.order;
     p.scale2 = a.sm_scale * kLog2e;
     p.sm_scale = a.sm_scale;
     p.inv_scale = 1.f / a.sm_scale;

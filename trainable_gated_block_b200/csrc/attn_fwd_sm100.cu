@@ -350,21 +350,22 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 tmem_ld32(tT + 64 * buf + 32, raw[1]);
                 tmem_wait_ld();
                 float x[64];
-                float mx = -INFINITY;
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // 4 independent chains
                 if (m.cur || !m.live) {
 #pragma unroll
                     for (int u = 0; u < 64; ++u) {
                         const bool live = m.live && u <= r_in;
                         x[u] = live ? fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2) : -INFINITY;
-                        mx = fmaxf(mx, x[u]);
+                        mx4[u & 3] = fmaxf(mx4[u & 3], x[u]);
                     }
                 } else {
 #pragma unroll
                     for (int u = 0; u < 64; ++u) {
                         x[u] = fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2);
-                        mx = fmaxf(mx, x[u]);
+                        mx4[u & 3] = fmaxf(mx4[u & 3], x[u]);
                     }
                 }
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 const float m_new = fmaxf(m_ref, mx);
                 const bool need = m_new > m_ref + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need) && k > 0) {
@@ -388,13 +389,15 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
                 uint32_t pk[32];
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};     // 4 independent chains
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const float p0 = fast_exp2(x[2 * e] - m_use);
                     const float p1 = fast_exp2(x[2 * e + 1] - m_use);
-                    l += p0 + p1;
+                    l4[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
+                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 tmem_st32(tT + 64 * buf, pk);
                 tmem_wait_st();
                 tc_fence_before();

@@ -149,13 +149,14 @@ struct Item {
 
 __device__ __forceinline__ Item item_of(const Params& p, int id) {
     Item it;
-    const int per_i = p.B * p.Hkv * p.ntile;
-    it.i = p.NQB - 1 - id / per_i;          // longest items first
-    int r = id % per_i;
+    // head by head (the CTAs working at the same time share one head's K/V in
+    // L2), query blocks from the last (longest items) down, then the tile
+    const int per_bh = p.NQB * p.ntile;
+    const int bh = id / per_bh, r = id % per_bh;
+    it.i = p.NQB - 1 - r / p.ntile;
     it.t = r % p.ntile;
-    r /= p.ntile;
-    it.h = r % p.Hkv;
-    it.b = r / p.Hkv;
+    it.h = bh % p.Hkv;
+    it.b = bh / p.Hkv;
     it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
     it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));
     it.nb = it.c + 1;
@@ -853,37 +854,46 @@ __global__ void __launch_bounds__(256) dot_rows_kernel(const __nv_bfloat16* __re
     }
 }
 
-// Sorts the dk/dv items (b, h, j) by decreasing step count (the length of
-// block j's reverse list) into `order`: 64 buckets of equal width, counted,
-// scanned by one warp and scattered; the order inside a bucket is arbitrary
-// (every item is computed on its own, so results do not depend on it).
-constexpr int kOrderBuckets = 64;
-__global__ void __launch_bounds__(1024) dkv_order_kernel(const int32_t* __restrict__ rcount, int n, int NQB,
+// Orders the dk/dv items (b, h, j): head by head (b, h ascending, so the CTAs
+// working at the same time share one head's Q/dO in L2), and inside a head by
+// decreasing step count (the length of block j's reverse list, `bpb` buckets
+// of equal width per head), so that the snake deal in dkv_kernel balances the
+// CTAs. Counted per bucket, scanned by one warp, scattered; the order inside
+// a bucket is arbitrary (every item is computed on its own, so results do not
+// depend on it).
+constexpr int kOrderMaxBuckets = 8192;
+__global__ void __launch_bounds__(1024) dkv_order_kernel(const int32_t* __restrict__ rcount, int n, int NQB, int bpb,
                                                          int32_t* __restrict__ order) {
-    __shared__ int cnt[kOrderBuckets], start[kOrderBuckets];
-    if (threadIdx.x < kOrderBuckets) cnt[threadIdx.x] = 0;
+    __shared__ int cnt[kOrderMaxBuckets];
+    const int nb = (n / NQB) * bpb;
+    for (int c = threadIdx.x; c < nb; c += blockDim.x) cnt[c] = 0;
     __syncthreads();
     auto bucket = [&](int id) {
-        const int j = id % NQB;
+        const int j = id % NQB, bh = id / NQB;
         const int c = max(1, min(rcount[id], NQB - j));      // steps of item id, 1..NQB
-        return (kOrderBuckets - 1) - (int)((long long)(c - 1) * kOrderBuckets / NQB);   // 0: largest
+        return bh * bpb + (bpb - 1) - (int)((long long)(c - 1) * bpb / NQB);
     };
     for (int id = threadIdx.x; id < n; id += blockDim.x) atomicAdd(&cnt[bucket(id)], 1);
     __syncthreads();
-    if (threadIdx.x < 32) {                                   // exclusive scan over the buckets
-        const int l = threadIdx.x;
-        const int a = cnt[2 * l], b = cnt[2 * l + 1];
-        int s = a + b;
+    if (threadIdx.x < 32) {                                   // exclusive scan: lane l owns a chunk of buckets
+        const int l = threadIdx.x, per = (nb + 31) / 32, lo = min(nb, l * per), hi = min(nb, lo + per);
+        int sum = 0;
+        for (int c = lo; c < hi; ++c) sum += cnt[c];
+        int incl = sum;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, s, d);
-            if (l >= d) s += t;
+            const int t = __shfl_up_sync(0xffffffffu, incl, d);
+            if (l >= d) incl += t;
         }
-        start[2 * l] = s - (a + b);
-        start[2 * l + 1] = s - b;
+        int run = incl - sum;
+        for (int c = lo; c < hi; ++c) {
+            const int v = cnt[c];
+            cnt[c] = run;
+            run += v;
+        }
     }
     __syncthreads();
-    for (int id = threadIdx.x; id < n; id += blockDim.x) order[atomicAdd(&start[bucket(id)], 1)] = id;
+    for (int id = threadIdx.x; id < n; id += blockDim.x) order[atomicAdd(&cnt[bucket(id)], 1)] = id;
 }
 
 __global__ void rev_fill_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int rows, int NQB,
@@ -978,7 +988,11 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
                                                                   (const __nv_bfloat16*)bw.dout, drows, a.S, a.Hq, ws.Dr);
     rev_fill_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(a.idx, a.cnt, bhq, NQB, a.K, ws.slotmap);
     rev_list_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(ws.slotmap, bhq, NQB, ws.rlist, ws.rcount);
-    dkv_order_kernel<<<1, 1024, 0, st>>>(ws.rcount, bhq, NQB, ws.order);
+    // buckets per head: 64, fewer when there are more than 128 (batch, KV head) pairs
+    const int n_bh = a.B * a.Hkv;
+    const int bpb = n_bh * 64 <= kOrderMaxBuckets ? 64 : (n_bh <= kOrderMaxBuckets ? kOrderMaxBuckets / n_bh : 0);
+    if (bpb == 0) return cudaErrorInvalidValue;
+    dkv_order_kernel<<<1, 1024, 0, st>>>(ws.rcount, bhq, NQB, bpb, ws.order);
     count_launches(4);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

@@ -8,7 +8,7 @@
 // Work item = (batch b, KV head h, query block i, head group tg): up to two
 // 128-row Q tiles, each tile = 2 query heads x the 64 rows of block i. All
 // query heads of a GQA group share the kept blocks, so one K/V block feeds
-// both Q tiles. Persistent grid; items in order of decreasing cost.
+// both Q tiles. Persistent grid; items head by head, longest first within a head.
 //
 // One step = one kept block (64 keys). Warp roles (352 threads):
 //   warp 0      TMA producer: the Q tiles once per item, then K and V of one
@@ -109,13 +109,14 @@ struct Item {
 
 __device__ __forceinline__ Item item_of(const Params& p, int id) {
     Item it;
-    const int per_i = p.B * p.Hkv * p.ntg;
-    it.i = p.NQB - 1 - id / per_i;
-    int r = id % per_i;
+    // head by head (the CTAs working at the same time share one head's K/V in
+    // L2), query blocks from the last (longest items) down, then the head group
+    const int per_bh = p.NQB * p.ntg;
+    const int bh = id / per_bh, r = id % per_bh;
+    it.i = p.NQB - 1 - r / p.ntg;
     it.tg = r % p.ntg;
-    r /= p.ntg;
-    it.h = r % p.Hkv;
-    it.b = r / p.Hkv;
+    it.h = bh % p.Hkv;
+    it.b = bh / p.Hkv;
     it.nt = (4 * it.tg + 2 < p.G) ? 2 : 1;
     it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
     it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));

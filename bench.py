@@ -90,6 +90,20 @@ def select_bytes(nh_total, rows, K):
 
 
 # ---------------------------------------------------------------------------
+# DRAM bytes (read + write) per call of each entry point, summed over its kernels,
+# from one `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` capture of
+# run_once on the workload (profiles/dram_traffic_qwen3-8b-32k.md); to be
+# retaken whenever one of those kernels changes.
+# ---------------------------------------------------------------------------
+DRAM_TRAFFIC = {
+    "qwen3-8b-32k": {
+        "sas_attn_fwd": 405804800 + 236452864,
+        "sas_attn_bwd": (684000768 + 238927872) + (4346328320 + 128374016) + (536907008 + 3521024),
+    },
+}
+
+
+# ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 
@@ -261,8 +275,9 @@ def run_ours(a):
     }
     dom = max(("fwd", "bwd", "decode", "select"), key=lambda n: part_ms[n])
     kd = kernels[dom]
+    traffic = DRAM_TRAFFIC.get(pc.name, {}).get(f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}")
     roofline = dict(bound=kd["bound"], achieved=round(kd["achieved"], 3), peak=kd["peak"], unit=kd["unit"],
-                    frac=round(kd["frac"], 4), traffic=None, kernel=f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}",
+                    frac=round(kd["frac"], 4), traffic=traffic, kernel=f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}",
                     peak_note=f"{tag} ({tnote if kd['bound'] == 'tensor' else 'HBM copy'})")
 
     e2e = None

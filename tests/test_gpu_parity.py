@@ -203,6 +203,21 @@ def _reverse(idx, cnt, b, h, j):
 @pytest.mark.parametrize("name", ["qwen3-4b-8k", "qwen3-8b-32k", "qwen3-14b-2x32k"])
 def test_full_workload_sampled(name):
     cfg = inputs.workload(name)
+    NQB = cfg.NQB
+    rnd = random.Random(cfg.seed)
+    _sampled_parity(cfg, [0, 1, NQB // 2, NQB - 1, rnd.randrange(NQB)])
+
+
+def test_mixed_tile_items_sampled():
+    """GQA group of 10: head groups of 4, 4 and 2 heads, so the forward's items alternate
+    between two Q tiles and one on the same CTA (384 items over a 148-CTA grid). Query blocks
+    0, 1, 15 and 64 are processed after an item with an idle tile on their CTA; 100 and 127
+    are first items."""
+    cfg = inputs.PrefillConfig("g10-mixed", "bf16", 1, 8192, 10, 1, 128, 8, "normal", 1.0, seed=21)
+    _sampled_parity(cfg, [0, 1, 15, 64, 100, 127])
+
+
+def _sampled_parity(cfg, rows):
     x = inputs.make_prefill(cfg)
     xd = _dev(x)
     NQB, G, D = cfg.NQB, cfg.G, cfg.D
@@ -214,10 +229,9 @@ def test_full_workload_sampled(name):
     torch.cuda.synchronize()
     sas.get_error_flag()
     idx, cnt, lg, _ = _select_checks(x["s"], cfg.K, gsel, O.prefill_history(NQB))
-    rnd = random.Random(cfg.seed)
+    rnd = random.Random(cfg.seed + 1)
     b = cfg.B - 1
     h = rnd.randrange(cfg.Hkv)
-    rows = [0, 1, NQB // 2, NQB - 1, rnd.randrange(NQB)]
     stripes = [(b, h * G + g, i) for i in rows for g in range(G)]
     ro, rlse = O.attn_fwd(x["q"], x["k"], x["v"], idx, cnt, lg, sc, stripes=stripes)
     rdq, _, _, rds, _ = O.attn_bwd(x["q"], x["k"], x["v"], x["do"], idx, cnt, lg, x["s"], sc, stripes=stripes)

@@ -18,7 +18,10 @@
 //               at a bounded rate, so each tile has its own. S_t = Q_t K^T
 //               into one of two S buffers per tile, O_t += P_t V with P read
 //               from TMEM. S of step j+2 is issued as soon as PV of step j is,
-//               so the softmax of step j+1 never waits for an MMA.
+//               so the softmax of step j+1 never waits for an MMA. On an
+//               item with one Q tile the idle issuer still waits for each Q
+//               and K/V phase and releases it, so it never falls two phases
+//               behind those barriers.
 //   warps 2-5   softmax of Q tile 0, warps 6-9 of tile 1: one row per thread
 //               (one TMEM lane); logits = sm_scale q.k + log-gate in the log2
 //               domain, causal mask on the diagonal block, running max/sum;
@@ -262,15 +265,23 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             bool ok = true;
             for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
                 const Item it = item_of(p, id);
-                if (t >= it.nt) {                       // tile 1 idle: tile 0's issuer arrives for it
-                    kv_it += it.nb;
-                    ++q_it;
-                    continue;
-                }
-                // arrivals this issuer owes the stage / Q barriers (2 when it is alone)
-                const int owe = (it.nt == 1) ? 2 : 1;
                 if (!(ok = mbar_wait(&bars->q_full, q_it & 1, abort, p.status))) break;
                 ++q_it;
+                if (t >= it.nt) {
+                    // Tile 1 idle: still wait every phase of the shared Q and K/V barriers and
+                    // release it at once, so that this issuer never falls two phases behind (a
+                    // parity wait on a barrier two phases ahead would pass on the wrong phase).
+                    for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
+                        const int st = kv_it % kNS;
+                        const uint32_t par = (kv_it / kNS) & 1;
+                        if (!(ok = mbar_wait(&bars->k_full[st], par, abort, p.status) &&
+                                   mbar_wait(&bars->v_full[st], par, abort, p.status)))
+                            break;
+                        if (k + 1 == it.nb) mbar_arrive(&bars->q_empty);
+                        mbar_arrive(&bars->kv_empty[st]);
+                    }
+                    continue;
+                }
                 tc_fence_after();
                 // prologue: S of the first two steps
                 for (int k = 0; k < 2 && k < it.nb && ok; ++k) {
@@ -280,8 +291,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     issue_s(g % kNS, k & 1);
                 }
                 if (!ok) break;
-                if (it.nb <= 2)
-                    for (int c = 0; c < owe; ++c) mma_commit(&bars->q_empty);
+                if (it.nb <= 2) mma_commit(&bars->q_empty);
                 for (int k = 0; k < it.nb && ok; ++k, ++kv_it) {
                     const int st = kv_it % kNS;
                     const int buf = k & 1;
@@ -306,9 +316,8 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         tc_fence_after();
                         issue_s(g2 % kNS, buf);
                     }
-                    if (k + 3 == it.nb)
-                        for (int c = 0; c < owe; ++c) mma_commit(&bars->q_empty);
-                    for (int c = 0; c < owe; ++c) mma_commit(&bars->kv_empty[st]);
+                    if (k + 3 == it.nb) mma_commit(&bars->q_empty);
+                    mma_commit(&bars->kv_empty[st]);
                     // publish PV completion: the softmax waits for it only when it
                     // rescales O and at the end of the item
                     if (!(ok = mbar_wait(&bars->o_done[t], pv_n & 1, abort, p.status))) break;

@@ -42,6 +42,8 @@ constexpr int kWarps = 3;                          // consumer warps
 constexpr int kThreads = (kWarps + 1) * 32;        // + one producer warp
 constexpr int kStages = 2 * kWarps;                // warp w owns stages w and w + kWarps
 constexpr uint32_t kBoxBytes = 64 * 128;           // TMA box: 64 rows x 64 dims (128 B)
+constexpr int kShortRows = 8;                      // short box (one 128-byte swizzle period) for a partial block
+constexpr uint32_t kShortBytes = kShortRows * 128;
 constexpr uint32_t kTileBytes = 2 * kBoxBytes;     // one (page, head) tile of K or V
 constexpr uint32_t kStageBytes = 2 * kTileBytes;
 constexpr uint32_t kOffMo = kStages * kStageBytes;                 // merge scratch: o [warp][8][D]
@@ -124,7 +126,8 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const Params p) {
+decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+              const __grid_constant__ CUtensorMap map_k8, const __grid_constant__ CUtensorMap map_v8, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* mo = reinterpret_cast<float*>(smem + kOffMo);
@@ -147,28 +150,35 @@ decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__
 
     const long long v0 = slot_begin(blockIdx.x, p.V, p.grid), v1 = slot_begin(blockIdx.x + 1, p.V, p.grid);
     const int Kp1 = p.K + 1;
+    // the combine kernel may be scheduled now (it waits for this grid to finish)
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == kWarps) {
         // ----------------------------------------------------------- producer
         // The 32 lanes resolve 32 block slots at a time (selection entry, page,
         // gate: dependent loads, done in parallel); lane 0 then issues the
-        // copies of the kept ones in slot order.
+        // copies of the kept ones in slot order. The next batch is resolved
+        // once the ring is full, while its copies are in flight, so the ring
+        // does not drain during those loads.
         if (lane == 0) {
             prefetch_tensormap(&map_k);
             prefetch_tensormap(&map_v);
+            prefetch_tensormap(&map_k8);
+            prefetch_tensormap(&map_v8);
         }
-        uint32_t it = 0;
-        bool ok_run = true;
-        for (long long base = v0; base < v1 && ok_run; base += 32) {
+        struct Slot {
+            bool use;
+            int row0;
+            float bias, nvalid;
+        };
+        auto resolve = [&](long long base) {
             const long long v = base + lane;
-            bool use = false;
-            int row0 = -1;
-            float bias = 0.f, nvalid = 0.f;
+            Slot s{false, -1, 0.f, 0.f};
             if (v < v1) {
                 const int item = (int)(v / Kp1), t = (int)(v % Kp1);
                 const ItemInfo inf = item_info(p, item, true);
                 if (inf.ok && t <= inf.n_sel) {
-                    use = true;
+                    s.use = true;
                     const bool cur = (t == inf.n_sel);
                     const long long srow = (long long)item * p.K + t;
                     const int j = cur ? inf.c : p.idx[srow];
@@ -177,27 +187,49 @@ decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__
                         page = p.page_table[(long long)inf.n * p.max_pages + j];
                     const bool ok = page >= 0 && page < p.num_pages;
                     if (!ok) flag_status(p.status, kStatusBadData);
-                    bias = cur ? 0.f : p.log_gate[srow] * kLog2e;
-                    nvalid = ok ? (float)(cur ? inf.L - inf.c * kBlock : kBlock) : 0.f;
-                    row0 = ok ? (page * p.Hkv + inf.h) * kBlock : -1;   // < 2^31 (checked on the host)
+                    s.bias = cur ? 0.f : p.log_gate[srow] * kLog2e;
+                    s.nvalid = ok ? (float)(cur ? inf.L - inf.c * kBlock : kBlock) : 0.f;
+                    s.row0 = ok ? (page * p.Hkv + inf.h) * kBlock : -1;   // < 2^31 (checked on the host)
                 }
             }
-            unsigned todo = __ballot_sync(0xffffffffu, use);
+            return s;
+        };
+        uint32_t it = 0;
+        bool ok_run = true;
+        Slot cur = resolve(v0);
+        for (long long base = v0; base < v1 && ok_run; base += 32) {
+            const bool more = base + 32 < v1;
+            Slot nxt{false, -1, 0.f, 0.f};
+            bool resolved = !more;
+            int issued = 0;
+            unsigned todo = __ballot_sync(0xffffffffu, cur.use);
             while (todo) {
                 const int b = __ffs(todo) - 1;
                 todo &= todo - 1;
-                const int rb = __shfl_sync(0xffffffffu, row0, b);
-                const float bb = __shfl_sync(0xffffffffu, bias, b);
-                const float nb = __shfl_sync(0xffffffffu, nvalid, b);
+                const int rb = __shfl_sync(0xffffffffu, cur.row0, b);
+                const float bb = __shfl_sync(0xffffffffu, cur.bias, b);
+                const float nb = __shfl_sync(0xffffffffu, cur.nvalid, b);
                 if (lane == 0) {
                     const int st = it % kStages;
                     if (!mbar_wait(&empty[st], ((it / kStages) & 1) ^ 1, abort, p.status)) {
                         ok_run = false;
                     } else {
                         meta[st] = make_float2(bb, nb);
-                        if (rb >= 0) {
+                        uint8_t* dst = smem + st * kStageBytes;
+                        const int nv = (int)nb;
+                        if (rb >= 0 && nv < kBlock) {
+                            // partial block (the current one): only the 8-row groups holding tokens
+                            const int ng = (nv + kShortRows - 1) / kShortRows;
+                            mbar_expect_tx(&full[st], (uint32_t)ng * 4 * kShortBytes);
+                            for (int g8 = 0; g8 < ng; ++g8)
+                                for (int a = 0; a < 2; ++a) {
+                                    const uint32_t off = a * kBoxBytes + g8 * kShortBytes;
+                                    tma_load_3d(dst + off, &map_k8, &full[st], a * 64, 0, rb + g8 * kShortRows);
+                                    tma_load_3d(dst + kTileBytes + off, &map_v8, &full[st], a * 64, 0,
+                                                rb + g8 * kShortRows);
+                                }
+                        } else if (rb >= 0) {
                             mbar_expect_tx(&full[st], kStageBytes);
-                            uint8_t* dst = smem + st * kStageBytes;
                             for (int a = 0; a < 2; ++a) {
                                 tma_load_3d(dst + a * kBoxBytes, &map_k, &full[st], a * 64, 0, rb);
                                 tma_load_3d(dst + kTileBytes + a * kBoxBytes, &map_v, &full[st], a * 64, 0, rb);
@@ -210,7 +242,13 @@ decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__
                 }
                 ok_run = __shfl_sync(0xffffffffu, ok_run, 0);
                 if (!ok_run) break;
+                if (!resolved && ++issued == kStages) {
+                    nxt = resolve(base + 32);
+                    resolved = true;
+                }
             }
+            if (!resolved) nxt = resolve(base + 32);
+            cur = nxt;
         }
         if (lane == 0 && *abort) {       // let the copies in flight land before the CTA exits
             volatile int no_abort = 0;
@@ -379,6 +417,9 @@ decode_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__
 __global__ void __launch_bounds__(kD)
 decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, int nslot, int Hq, int Hkv,
                       int G, int K, long long V, int grid, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+    // launched as a programmatic dependent of decode_kernel: its blocks may be
+    // resident before the decode grid ends; wait for that grid's writes here
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const long long row = blockIdx.x;          // n * Hq + hq
     const int d = threadIdx.x;
     const long long n = row / Hq;
@@ -436,8 +477,10 @@ cudaError_t launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t st)
     const Layout lay = layout(a.N, a.Hkv, a.K);
     float* part_o = static_cast<float*>(workspace);
     float* part_ml = part_o + (size_t)a.N * a.Hq * lay.nslot * kD;
-    CUtensorMap mk, mv;
-    if (!make_head_map(&mk, a.k_cache, cache_rows, 1, kD) || !make_head_map(&mv, a.v_cache, cache_rows, 1, kD))
+    CUtensorMap mk, mv, mk8, mv8;
+    if (!make_head_map(&mk, a.k_cache, cache_rows, 1, kD) || !make_head_map(&mv, a.v_cache, cache_rows, 1, kD) ||
+        !make_head_map(&mk8, a.k_cache, cache_rows, 1, kD, kShortRows) ||
+        !make_head_map(&mv8, a.v_cache, cache_rows, 1, kD, kShortRows))
         return cudaErrorInvalidValue;
     Params p;
     p.q = (const __nv_bfloat16*)a.q;
@@ -461,10 +504,23 @@ cudaError_t launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t st)
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
-    decode_kernel<<<lay.grid, kThreads, kSmem, st>>>(mk, mv, p);
+    decode_kernel<<<lay.grid, kThreads, kSmem, st>>>(mk, mv, mk8, mv8, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    decode_combine_kernel<<<a.N * a.Hq, kD, 0, st>>>(part_o, part_ml, lay.nslot, a.Hq, a.Hkv, G, a.K, lay.V,
-                                                      lay.grid, (__nv_bfloat16*)a.o, a.lse);
+    // programmatic dependent launch: the combine's blocks are placed while the
+    // decode grid drains, which removes the launch gap between the two kernels
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.N * a.Hq));
+    cfg.blockDim = dim3(kD);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, (const float*)part_o, (const float*)part_ml, lay.nslot, a.Hq,
+                           a.Hkv, G, a.K, lay.V, lay.grid, (__nv_bfloat16*)a.o, a.lse);
+    if (e != cudaSuccess) return e;
     count_launches(2);
     return cudaGetLastError();
 }

@@ -311,6 +311,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // TMA map of a [rows, H, D] bf16 tensor as 3-D (D, H, rows): 64 x 1 x 64
 // boxes, 128-byte swizzle (tma_maps.cu).
-bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D);
+bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D, int box_rows = 64);
 
 }  // namespace sas

@@ -22,13 +22,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// [rows, H, D] bf16 viewed as 3-D (D, H, rows); 64 x 1 x 64 boxes, 128B swizzle.
-bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D) {
+// [rows, H, D] bf16 viewed as 3-D (D, H, rows); 64 x 1 x box_rows boxes, 128B swizzle.
+bool make_head_map(CUtensorMap* map, const void* base, long long rows, int H, int D, int box_rows) {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -61,6 +61,38 @@ def _peaks():
 
 
 # ---------------------------------------------------------------------------
+# replicas: one process per GPU, no collective in the data path
+# ---------------------------------------------------------------------------
+
+def rank_env():
+    """(world size, rank, local rank) as torchrun sets them; one process without it."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(base, rank):
+    """Each rank runs its own replica of the workload on its own seeded inputs."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(vals, dist, device):
+    """Element-wise max of per-rank timings over the process group (the slowest
+    rank sets the job's time); the values unchanged in a single process."""
+    vals = [float(v) for v in vals]
+    if dist is None or not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return vals
+    import torch
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def weak_tflops(world, flops_per_replica, ms):
+    """Whole-job throughput: the flops of every replica over the slowest rank's time."""
+    return world * flops_per_replica / (ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # work counts (algorithmic)
 # ---------------------------------------------------------------------------
 
@@ -157,9 +189,7 @@ def run_ours(a):
 
     from trainable_gated_block_b200 import build, inputs, sas
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
@@ -174,8 +204,8 @@ def run_ours(a):
 
     pc = inputs.workload(a.prefill)
     dc = inputs.workload(a.decode)
-    px = inputs.make_prefill(pc, seed=pc.seed + 1000 * rank)
-    dx = inputs.make_decode(dc, seed=dc.seed + 1000 * rank)
+    px = inputs.make_prefill(pc, seed=replica_seed(pc.seed, rank))
+    dx = inputs.make_decode(dc, seed=replica_seed(dc.seed, rank))
     P = {k: v.to(dev) for k, v in px.items()}
     Dd = {k: v.to(dev) for k, v in dx.items()}
     sc_p = 1.0 / math.sqrt(pc.D)
@@ -238,16 +268,14 @@ def run_ours(a):
     part_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / a.steps for i, n in enumerate(names)}
     prefill_ms = part_ms["select"] + part_ms["fwd"] + part_ms["bwd"]
     dec_ms = part_ms["dselect"] + part_ms["decode"]
-    if world > 1:
-        t = torch.tensor([total_ms, prefill_ms, dec_ms] + [part_ms[n] for n in names], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, prefill_ms, dec_ms = float(t[0]), float(t[1]), float(t[2])
-        part_ms = {n: float(t[3 + i]) for i, n in enumerate(names)}
+    t = max_over_ranks([total_ms, prefill_ms, dec_ms] + [part_ms[n] for n in names], dist, dev)
+    total_ms, prefill_ms, dec_ms = t[0], t[1], t[2]
+    part_ms = {n: t[3 + i] for i, n in enumerate(names)}
 
     tiles = prefill_tiles(pc)
     unit_flops = 64 * 64 * pc.D
     flops_fb = 14 * unit_flops * tiles
-    tflops = world * flops_fb / (prefill_ms * 1e-3) / 1e12
+    tflops = weak_tflops(world, flops_fb, prefill_ms)
     bwd_tf = 10 * unit_flops * tiles / (part_ms["bwd"] * 1e-3) / 1e12
     fwd_tf = 4 * unit_flops * tiles / (part_ms["fwd"] * 1e-3) / 1e12
     dec_gbs = dec_bytes / (part_ms["decode"] * 1e-3) / 1e9
@@ -367,12 +395,9 @@ def run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, wo
     sas.get_error_flag()
     pre = sum(e[0].elapsed_time(e[1]) for e in evs) / a.steps
     dec = sum(e[1].elapsed_time(e[2]) for e in evs) / a.steps
-    if world > 1:
-        t = torch.tensor([pre, dec], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        pre, dec = float(t[0]), float(t[1])
+    pre, dec = max_over_ranks([pre, dec], dist, dev)
     d2h = sum(t.numel() * t.element_size() for t in outs.values())
-    return dict(value=round(world * flops_fb / (pre * 1e-3) / 1e12, 3), unit="TFLOPS",
+    return dict(value=round(weak_tflops(world, flops_fb, pre), 3), unit="TFLOPS",
                 h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
                 ms_prefill=round(pre, 3), ms_decode=round(dec, 3),
                 decode_tokens_per_s=round(world * dc.N / (dec * 1e-3), 1))
@@ -430,8 +455,8 @@ def cpu_baseline(pc, px, budget_s):
 
 
 def run_reference(a):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    _, rank, _ = rank_env()
+    if rank != 0:          # the oracle runs once, on rank 0; the other ranks exit without work
         return
     from trainable_gated_block_b200 import inputs
     pc = inputs.workload(a.prefill)

@@ -206,6 +206,19 @@ sas_status sas_decode_paged_noalloc(const void *q, const void *k_cache, const vo
                                     const float *log_gate, float sm_scale, void *o, float *lse,
                                     void *stream);
 
+/*
+ * sas_selftest_bounded_wait - fault injection for the bounded waits, with no
+ * GPU fault (no counterpart on the SAS pages: it tests this library's failure
+ * detection). Enqueues on `stream` one single-warp kernel that waits, with
+ * the bounded mbarrier wait every kernel of the library uses, on a barrier
+ * that nothing ever arrives on. The wait gives up after its budget (about 2 s
+ * of SM clocks), records a timeout in the device status word and the kernel
+ * returns; the next sas_get_error_flag on the device reports (and clears)
+ * SAS_ERR_TIMEOUT, and the context stays usable.
+ * Returns SAS_OK once the kernel is enqueued, SAS_ERR_CUDA if it is not.
+ */
+sas_status sas_selftest_bounded_wait(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -186,6 +186,21 @@ def test_bad_indices_are_flagged_not_followed():
     sas.get_error_flag()             # cleared
 
 
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    """Failure detection without a GPU fault: a wait that can never complete gives up on
+    its budget, the host reads SAS_ERR_TIMEOUT once, and the next call runs normally."""
+    sas.get_error_flag()                 # nothing pending
+    sas.selftest_bounded_wait()
+    with pytest.raises(sas.SasError) as e:
+        sas.get_error_flag()
+    assert e.value.code == sas.SAS_ERR_TIMEOUT
+    sas.get_error_flag()                 # reported once, then cleared
+    s = torch.from_numpy(np.random.default_rng(11).standard_normal((1, 2, 40, 40)).astype(np.float32))
+    gsel = sas.select(_poisoned(s).cuda(), 5)
+    sas.get_error_flag()
+    _select_checks(s, 5, gsel, O.prefill_history(40))
+
+
 # ---------------------------------------------------------------------------
 # full workload sizes, sampled
 # ---------------------------------------------------------------------------

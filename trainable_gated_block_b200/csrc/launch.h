@@ -62,4 +62,7 @@ struct DecodeArgs {
 size_t decode_workspace(int N, int Hq, int Hkv, int D, int K);
 cudaError_t launch_decode(const DecodeArgs& d, void* workspace, cudaStream_t st);
 
+// One warp waiting (bounded) on a barrier nothing arrives on: records a timeout in *status.
+cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t st);
+
 }  // namespace sas

@@ -202,4 +202,11 @@ sas_status sas_decode_paged(const void* q, const void* k_cache, const void* v_ca
     return e == cudaSuccess ? ok() : cuda_fail(e, "sas_decode_paged");
 }
 
+sas_status sas_selftest_bounded_wait(void* stream) {
+    int* st = status_ptr();
+    if (!st) return fail(SAS_ERR_CUDA, "sas_selftest_bounded_wait: no CUDA device");
+    cudaError_t e = sas::launch_bounded_wait_selftest(st, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "sas_selftest_bounded_wait");
+}
+
 }  // extern "C"

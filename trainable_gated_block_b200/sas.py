@@ -39,6 +39,7 @@ SIGNATURES = {
                               _P, _P, _P, _F, _P, _P, _P, _Z, _P]),
     "sas_decode_paged_noalloc": (_I, [_P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                       _P, _P, _P, _F, _P, _P, _P]),
+    "sas_selftest_bounded_wait": (_I, [_P]),
 }
 
 
@@ -102,6 +103,13 @@ def kernel_launches() -> int:
 def get_error_flag(stream=None):
     """Synchronise the stream and raise if a kernel flagged bad data or a timeout."""
     _check(lib().sas_get_error_flag(_stream(stream)))
+
+
+def selftest_bounded_wait(stream=None):
+    """Enqueue the library's bounded-wait fault injection: a kernel whose wait can never
+    complete gives up after its budget (about 2 s) and the next get_error_flag raises
+    SasError with SAS_ERR_TIMEOUT."""
+    _check(lib().sas_selftest_bounded_wait(_stream(stream)))
 
 
 def select(s, K: int, kv_len=None, block_size: int = 64):

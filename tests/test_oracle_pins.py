@@ -38,6 +38,20 @@ MUTANTS = {
     "Dr_dropped": ("dS = P * (dP - Dr)", "dS = P * dP"),
     "decode_current_block_short": ("bias[c * BLOCK:L] = 0.0", "bias[c * BLOCK:L - 1 + (L - 1 == c * BLOCK)] = 0.0"),
     "decode_history_includes_current": ("return (_i64(kv_len) - 1) // BLOCK", "return (_i64(kv_len) + BLOCK - 1) // BLOCK"),
+    "prefill_history_includes_current": ("return np.arange(n_rows, dtype=np.int64)",
+                                         "return np.arange(n_rows, dtype=np.int64) + 1"),
+    "dq_missing_scale": ("dq[b, rs, hq, :] = sm_scale * (dS @ Kh)", "dq[b, rs, hq, :] = (dS @ Kh)"),
+    "topk_lowest_scores": ("np.lexsort((np.arange(nh), -s_row))", "np.lexsort((np.arange(nh), s_row))"),
+    "fwd_lse_missing_max": ("return P @ Vh, m[:, 0] + np.log(Z[:, 0]), P, L", "return P @ Vh, np.log(Z[:, 0]), P, L"),
+    "jacobian_softmax_over_selected": ("p = np.exp(row - logsumexp(row))",
+                                       "p = np.exp(row - logsumexp(row[sel])) * np.isin(np.arange(i), sel)"),
+    "decode_gate_sign": ("bias[j * BLOCK:(j + 1) * BLOCK] = log_gate[n, h, slot]",
+                         "bias[j * BLOCK:(j + 1) * BLOCK] = -log_gate[n, h, slot]"),
+    "decode_page_offset": ("off = pos % BLOCK", "off = (pos + 1) % BLOCK"),
+    "decode_lse_missing_max": ("lse[n, hq] = m + math.log(z)", "lse[n, hq] = math.log(z)"),
+    "dv_half": ("dv[b, :, h, :] += P.T @ dOi", "dv[b, :, h, :] += 0.5 * (P.T @ dOi)"),
+    "selection_left_in_score_order": ("return sorted(int(j) for j in order[:min(K, nh)])",
+                                      "return [int(j) for j in order[:min(K, nh)]]"),
 }
 
 

@@ -416,8 +416,11 @@ def _blas_threads():
         return 1
 
 
-def _oracle_stripes(pc, px, budget_s, max_stripes=10**9):
-    """Time oracle forward+backward stripes of the workload until the budget is spent."""
+def _oracle_stripes(pc, px, budget_s, max_stripes=10**9, parts=None):
+    """Time oracle forward+backward stripes of the workload until the budget is spent.
+
+    Returns (attended-tile flops, stripes, seconds of fwd+bwd); if a dict is
+    given as ``parts``, the seconds of select, fwd and bwd are added to it."""
     import numpy as np
 
     from oracle import sas_oracle as O
@@ -433,25 +436,37 @@ def _oracle_stripes(pc, px, budget_s, max_stripes=10**9):
         if t_spent >= budget_s or n >= max_stripes:
             break
         s1 = s[:1, :1, i:i + 1, :]
+        t_sel = time.perf_counter()
         idx1, cnt1, lg1, _ = O.select(s1, pc.K, np.array([[i]]))
+        t_sel = time.perf_counter() - t_sel
         idx = np.full((1, 1, pc.NQB, pc.K), -1, dtype=np.int32)
         cnt = np.zeros((1, 1, pc.NQB), dtype=np.int32)
         lg = np.full((1, 1, pc.NQB, pc.K), -np.inf)
         idx[0, 0, i], cnt[0, 0, i], lg[0, 0, i] = idx1[0, 0, 0], cnt1[0, 0, 0], lg1[0, 0, 0]
         t0 = time.perf_counter()
         O.attn_fwd(q, k, v, idx, cnt, lg, sc, stripes=[(0, 0, i)])
+        t1 = time.perf_counter()
         O.attn_bwd(q, k, v, do, idx, cnt, lg, s, sc, stripes=[(0, 0, i)])
-        t_spent += time.perf_counter() - t0
+        t2 = time.perf_counter()
+        t_spent += t2 - t0
+        if parts is not None:
+            for name, dt in (("select", t_sel), ("fwd", t1 - t0), ("bwd", t2 - t1)):
+                parts[name] = parts.get(name, 0.0) + dt
         flops += 14 * 64 * 64 * pc.D * (int(cnt[0, 0, i]) + 1)
         n += 1
     return flops, n, t_spent
 
 
 def cpu_baseline(pc, px, budget_s):
-    flops, n, t = _oracle_stripes(pc, px, budget_s)
+    parts = {}
+    flops, n, t = _oracle_stripes(pc, px, budget_s, parts=parts)
     return dict(value=flops / t / 1e12, unit="TFLOPS", cores=_blas_threads(), kind="oracle",
                 sample=f"fp64 oracle forward+backward of {n} 64-row stripes (batch 0, head 0) of the "
-                       f"{pc.name} workload, {t:.1f} s, counted as attended-tile flops")
+                       f"{pc.name} workload, {t:.1f} s, counted as attended-tile flops",
+                parts_s={k: round(v, 3) for k, v in parts.items()},
+                fwd_tflops=(4 / 14) * flops / parts["fwd"] / 1e12 if parts.get("fwd") else None,
+                bwd_tflops=(10 / 14) * flops / parts["bwd"] / 1e12 if parts.get("bwd") else None,
+                affinity_cores=len(os.sched_getaffinity(0)))
 
 
 def run_reference(a):

@@ -5,6 +5,8 @@ inputs, no collective in the data path); the only cross-rank step is the max
 of the timings, so that the slowest rank sets the job's time. Here two
 ``gloo`` ranks run that step, and a two-rank torchrun launch runs the
 reference arm, which must print one line from rank 0 and none elsewhere.
+The bench's CPU-baseline leg, which runs on the host alone, is checked here
+too.
 """
 import json
 import os
@@ -101,3 +103,14 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_cpu_baseline_line_on_cpu():
+    """The bench's CPU-baseline leg (the fp64 oracle on a bounded sample) runs on the host alone."""
+    cfg = inputs.workload("qwen3-4b-8k")
+    x = inputs.make_prefill(cfg)
+    cb = bench.cpu_baseline(cfg, x, 0.5)
+    assert cb["kind"] == "oracle" and cb["unit"] == "TFLOPS" and cb["value"] > 0
+    assert cb["cores"] >= 1 and cb["affinity_cores"] >= 1
+    assert set(cb["parts_s"]) == {"select", "fwd", "bwd"} and all(v >= 0 for v in cb["parts_s"].values())
+    assert cb["fwd_tflops"] > 0 and cb["bwd_tflops"] > 0

@@ -297,6 +297,33 @@ def decode(q, k_cache, v_cache, page_table, kv_len, idx, cnt, log_gate, sm_scale
 
 
 # ----------------------------------------------------------------------------
+# Stand-in selector scores: the step before select. The pages' selector
+# (AttnGate, SAS review §2.2) needs trained weights, so its scores are stood in
+# for by pooled attention logits: the mean of q over the 64 rows of block i and
+# the G query heads of KV head h, dotted with the mean of k[h] over the 64 rows
+# of block j, over sqrt(D), plus a given noise term (the random part is an
+# input, drawn by the caller).
+# ----------------------------------------------------------------------------
+
+def standin_scores(q, k, noise):
+    """s[b, h, i, j] = mean_{64 rows of block i, G heads of h}(q) . mean_{64 rows of block j}(k[:, :, h]) / sqrt(D)
+    + noise[b, h, i, j], in fp64. q [B,S,Hq,D], k [B,S,Hkv,D], noise [B,Hkv,NQB,NQB]; every
+    (i, j) is produced (select reads only j < i)."""
+    q, k, noise = _f64(q), _f64(k), _f64(noise)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    NQB = S // BLOCK
+    qp = q.reshape(B, NQB, BLOCK, Hkv, G, D).mean(axis=(2, 4))      # [B, NQB, Hkv, D]
+    kp = k.reshape(B, NQB, BLOCK, Hkv, D).mean(axis=2)              # [B, NQB, Hkv, D]
+    s = np.zeros((B, Hkv, NQB, NQB))
+    for b in range(B):
+        for h in range(Hkv):
+            s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)
+    return s + noise
+
+
+# ----------------------------------------------------------------------------
 # Work counts used to express throughput (not part of the method).
 # ----------------------------------------------------------------------------
 

@@ -433,8 +433,45 @@ def pin_decode_vs_prefill(O):
     assert G == 2
 
 
+def pin_standin_scores(O):
+    """Stand-in scores against explicit loops, a closed form and their invariances."""
+    B, S, Hq, Hkv, D = 2, 192, 6, 2, 8
+    G, NQB = Hq // Hkv, S // BLOCK
+    q = _rand((B, S, Hq, D), 31)
+    k = _rand((B, S, Hkv, D), 32)
+    noise = _rand((B, Hkv, NQB, NQB), 33)
+    s = O.standin_scores(q, k, noise)
+    # brute force: the two means summed element by element
+    ref = np.zeros((B, Hkv, NQB, NQB))
+    for b in range(B):
+        for h in range(Hkv):
+            for i in range(NQB):
+                for j in range(NQB):
+                    dot = 0.0
+                    for d in range(D):
+                        qm = sum(q[b, i * BLOCK + t, h * G + g, d] for t in range(BLOCK) for g in range(G)) / (BLOCK * G)
+                        km = sum(k[b, j * BLOCK + t, h, d] for t in range(BLOCK)) / BLOCK
+                        dot += qm * km
+                    ref[b, h, i, j] = dot / math.sqrt(D) + noise[b, h, i, j]
+    assert np.allclose(s, ref, rtol=1e-12, atol=1e-12)
+    # closed form: constant q = a, k = c gives a * c * D / sqrt(D) = a * c * sqrt(D)
+    sc = O.standin_scores(np.full((1, 128, 4, 16), 0.5), np.full((1, 128, 2, 16), -3.0), np.zeros((1, 2, 2, 2)))
+    assert np.allclose(sc, 0.5 * -3.0 * math.sqrt(16), rtol=1e-14)
+    # invariances: row order inside a block, and linearity in q
+    perm = np.random.default_rng(34).permutation(BLOCK)
+    qp = q.copy()
+    qp[:, BLOCK:2 * BLOCK] = q[:, BLOCK + perm]
+    assert np.allclose(O.standin_scores(qp, k, noise), s, rtol=1e-12, atol=1e-12)
+    assert np.allclose(O.standin_scores(2.0 * q, k, noise) - noise, 2.0 * (s - noise), rtol=1e-12, atol=1e-12)
+    # GQA map: query head hq pools into KV head hq // G only
+    q1 = np.zeros_like(q)
+    q1[:, :, G + 1, :] = q[:, :, G + 1, :]
+    s1 = O.standin_scores(q1, k, np.zeros_like(noise))
+    assert np.all(s1[:, 0] == 0.0) and np.any(s1[:, 1] != 0.0)
+
+
 ALL_PINS = [
     pin_topk_rank, pin_select_gates, pin_golden, pin_dense_equivalence, pin_block_diagonal,
     pin_general_sdpa, pin_bruteforce_loops, pin_finite_differences, pin_shift_invariance,
-    pin_sparsity, pin_probabilities, pin_decode_vs_sdpa, pin_decode_vs_prefill,
+    pin_sparsity, pin_probabilities, pin_decode_vs_sdpa, pin_decode_vs_prefill, pin_standin_scores,
 ]

@@ -52,6 +52,14 @@ MUTANTS = {
     "dv_half": ("dv[b, :, h, :] += P.T @ dOi", "dv[b, :, h, :] += 0.5 * (P.T @ dOi)"),
     "selection_left_in_score_order": ("return sorted(int(j) for j in order[:min(K, nh)])",
                                       "return [int(j) for j in order[:min(K, nh)]]"),
+    "standin_sum_not_mean": ("qp = q.reshape(B, NQB, BLOCK, Hkv, G, D).mean(axis=(2, 4))",
+                             "qp = q.reshape(B, NQB, BLOCK, Hkv, G, D).sum(axis=(2, 4))"),
+    "standin_heads_interleaved": ("qp = q.reshape(B, NQB, BLOCK, Hkv, G, D).mean(axis=(2, 4))",
+                                  "qp = q.reshape(B, NQB, BLOCK, G, Hkv, D).mean(axis=(2, 3))"),
+    "standin_scale_d": ("s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)",
+                        "s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / D"),
+    "standin_transposed": ("s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)",
+                           "s[b, h] = (kp[b, :, h, :] @ qp[b, :, h, :].T) / math.sqrt(D)"),
 }
 
 
@@ -73,3 +81,21 @@ def test_mutant_is_caught(name):
         except Exception:          # an assertion, or a crash the slip causes
             caught.append(pin.__name__)
     assert caught, f"no pin catches the planted mistake {name!r}"
+
+
+def test_workload_scores_are_the_standin_definition():
+    """The seeded 8k/32k workloads' scores are the oracle's stand-in scores plus the N(0,1)
+    noise drawn fourth (after q, k, v) from the workload's generator, rounded to fp32 once."""
+    import torch
+
+    from trainable_gated_block_b200 import inputs
+    cfg = inputs.PrefillConfig("standin-small", "bf16", 1, 512, 8, 2, 128, 4, "standin", seed=41)
+    x = inputs.make_prefill(cfg, with_do=False)
+    g = torch.Generator().manual_seed(41)
+    q = inputs._randn((1, 512, 8, 128), g, torch.bfloat16)
+    k = inputs._randn((1, 512, 2, 128), g, torch.bfloat16)
+    inputs._randn((1, 512, 2, 128), g, torch.bfloat16)            # v
+    noise = inputs._randn((1, 2, 8, 8), g, torch.float32)
+    assert torch.equal(q, x["q"]) and torch.equal(k, x["k"])
+    ref = sas_oracle.standin_scores(q, k, noise).astype("float32")
+    assert (ref == x["s"].numpy()).all()

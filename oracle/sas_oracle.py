@@ -23,7 +23,7 @@ Method (SAS review (paper.oopus.info), §2.1-§2.6; SAS abstract (fugumt.com)):
 * §2.6: the gradient of a block's gate is the sum of the logit gradients
   inside that block; it reaches the scores through the LSE Jacobian.
 
-Readings taken where the pages are silent (each listed in the design doc):
+Readings taken where the pages are silent:
 
 * the logits are ``sm_scale * q.k + log g``, sm_scale scaling q.k only;
 * history of query block i = blocks 0..i-1; block 0 has no history, no gate;
@@ -37,6 +37,17 @@ Readings taken where the pages are silent (each listed in the design doc):
 * decode: the query sits at position ``kv_len-1``; its current block is
   ``c = (kv_len-1)//64`` holding tokens ``64c..kv_len-1``; its history is
   blocks ``0..c-1``.
+* a prefill length S that is not a multiple of 64 ends in a partial block
+  ``ceil(S/64)-1`` of ``S - 64*(ceil(S/64)-1)`` tokens: it is a query block
+  like any other (its rows attend its own keys causally and its kept history
+  blocks), and as a history block of no later query block it is never
+  selected; the same rule as decode's partial current block.
+* a batch of sequences of different lengths (packed along the token axis,
+  sequence b holding tokens ``cu_seqlens[b]..cu_seqlens[b+1]-1``) is the
+  method applied to each sequence on its own; the per-block tensors (scores,
+  selection, ds) and the row LSE keep a padded ``[B, ..., max blocks]`` /
+  ``[B, Hq, max length]`` layout whose entries past a sequence's end are
+  padding.
 
 Parity pins for every function are in ``tests/test_oracle_pins.py``.
 """
@@ -136,19 +147,32 @@ def select(s, K: int, n_hist):
 # kept ungated (§2.4, g_0 = 1) under a causal mask.
 # ----------------------------------------------------------------------------
 
+def block_rows(i: int, S: int) -> slice:
+    """Token rows of block i in a sequence of S tokens (the last block may be partial)."""
+    return slice(i * BLOCK, min(S, (i + 1) * BLOCK))
+
+
+def n_blocks(S: int) -> int:
+    """Blocks of a sequence of S tokens, the last one possibly partial."""
+    return (S + BLOCK - 1) // BLOCK
+
+
 def stripe_bias(i: int, S: int, sel, gates) -> np.ndarray:
-    """Masked bias of the 64 query rows of block i over all S keys.
+    """Masked bias of the query rows of block i over all S keys.
 
     0 on the causal part of the current block, the block's log-gate on every
-    key of a selected history block, -inf everywhere else.
+    key of a selected history block, -inf everywhere else. Block i has 64
+    rows, or fewer when it is the last, partial block of the sequence.
     """
-    bias = np.full((BLOCK, S), NEG_INF)
+    rows = block_rows(i, S)
+    n = rows.stop - rows.start
+    bias = np.full((n, S), NEG_INF)
     for j, lg in zip(sel, gates):
         assert 0 <= j < i
         bias[:, j * BLOCK:(j + 1) * BLOCK] = lg
-    t = np.arange(BLOCK)[:, None]
-    u = np.arange(BLOCK)[None, :]
-    bias[:, i * BLOCK:(i + 1) * BLOCK] = np.where(u <= t, 0.0, NEG_INF)
+    t = np.arange(n)[:, None]
+    u = np.arange(n)[None, :]
+    bias[:, rows] = np.where(u <= t, 0.0, NEG_INF)
     return bias
 
 
@@ -158,12 +182,12 @@ def _row_selection(idx, cnt, log_gate, b, h, i):
 
 
 def fwd_stripe(q, k, v, idx, cnt, log_gate, sm_scale, b, hq, i):
-    """One 64-row stripe: returns (o [64,D], lse [64], P [64,S], L [64,S])."""
+    """One stripe (the n <= 64 rows of block i): returns (o [n,D], lse [n], P [n,S], L [n,S])."""
     S = q.shape[1]
     G = q.shape[2] // k.shape[2]
     h = hq // G
     sel, gates = _row_selection(idx, cnt, log_gate, b, h, i)
-    Qi = q[b, i * BLOCK:(i + 1) * BLOCK, hq, :]
+    Qi = q[b, block_rows(i, S), hq, :]
     Kh = k[b, :, h, :]
     Vh = v[b, :, h, :]
     L = sm_scale * (Qi @ Kh.T) + stripe_bias(i, S, sel, gates)
@@ -186,11 +210,11 @@ def attn_fwd(q, k, v, idx, cnt, log_gate, sm_scale, stripes=None):
     o = np.full((B, S, Hq, D), np.nan)
     lse = np.full((B, Hq, S), np.nan)
     if stripes is None:
-        stripes = [(b, hq, i) for b in range(B) for hq in range(Hq) for i in range(S // BLOCK)]
+        stripes = [(b, hq, i) for b in range(B) for hq in range(Hq) for i in range(n_blocks(S))]
     for b, hq, i in stripes:
         oi, li, _, _ = fwd_stripe(q, k, v, idx, cnt, log_gate, sm_scale, b, hq, i)
-        o[b, i * BLOCK:(i + 1) * BLOCK, hq, :] = oi
-        lse[b, hq, i * BLOCK:(i + 1) * BLOCK] = li
+        o[b, block_rows(i, S), hq, :] = oi
+        lse[b, hq, block_rows(i, S)] = li
     return o, lse
 
 
@@ -207,14 +231,14 @@ def attn_bwd(q, k, v, do, idx, cnt, log_gate, s, sm_scale, stripes=None):
     and dk/dv of a key block are exact when every stripe that attends it is
     listed. Returns dq, dk, dv (fp64, input layouts), ds fp64 [B,Hkv,NQB,NQB]
     (zero on j >= i) and gsum fp64 [B,Hkv,NQB,NQB] (the per-block gate
-    gradients dL/dlog g_ij, zero where j is not selected).
+    gradients dL/dlog g_ij, zero where j is not selected); NQB = ceil(S/64).
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     idx, cnt, log_gate, s = _i64(idx), _i64(cnt), _f64(log_gate), _f64(s)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
-    NQB = S // BLOCK
+    NQB = n_blocks(S)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -225,7 +249,7 @@ def attn_bwd(q, k, v, do, idx, cnt, log_gate, s, sm_scale, stripes=None):
     for b, hq, i in stripes:
         h = hq // G
         _, _, P, _ = fwd_stripe(q, k, v, idx, cnt, log_gate, sm_scale, b, hq, i)
-        rs = slice(i * BLOCK, (i + 1) * BLOCK)
+        rs = block_rows(i, S)
         Qi, dOi = q[b, rs, hq, :], do[b, rs, hq, :]
         Kh, Vh = k[b, :, h, :], v[b, :, h, :]
         dv[b, :, h, :] += P.T @ dOi
@@ -235,7 +259,7 @@ def attn_bwd(q, k, v, do, idx, cnt, log_gate, s, sm_scale, stripes=None):
         dq[b, rs, hq, :] = sm_scale * (dS @ Kh)
         dk[b, :, h, :] += sm_scale * (dS.T @ Qi)
         if i > 0:
-            gsum[b, h, i, :i] += dS[:, :i * BLOCK].reshape(BLOCK, i, BLOCK).sum(axis=(0, 2))
+            gsum[b, h, i, :i] += dS[:, :i * BLOCK].reshape(len(Qi), i, BLOCK).sum(axis=(0, 2))
         rows_done.add((b, h, i))
     ds = np.zeros((B, Hkv, NQB, NQB))
     for b, h, i in rows_done:
@@ -249,6 +273,78 @@ def attn_bwd(q, k, v, do, idx, cnt, log_gate, s, sm_scale, stripes=None):
         for m in sel:
             ds[b, h, i, m] += gsum[b, h, i, m]
     return dq, dk, dv, ds, gsum
+
+
+# ----------------------------------------------------------------------------
+# Batches of sequences of different lengths, packed along the token axis: the
+# method (SAS review §2.1-§2.6) applied to each sequence on its own.
+# ----------------------------------------------------------------------------
+
+def seq_bounds(cu_seqlens):
+    """(start, length) of every sequence of a packed batch."""
+    cu = _i64(cu_seqlens)
+    return [(int(cu[b]), int(cu[b + 1] - cu[b])) for b in range(len(cu) - 1)]
+
+
+def select_varlen(s, K: int, cu_seqlens):
+    """select() per sequence: s [B, Hkv, R, ld] with R >= the most blocks of any
+    sequence; row i of sequence b is a query block when i < ceil(len_b/64) and
+    padding otherwise (cnt 0, idx -1, log-gate -inf, lse_s -inf)."""
+    s = _f64(s)
+    B, H, R, _ = s.shape
+    idx = np.full((B, H, R, K), -1, dtype=np.int32)
+    cnt = np.zeros((B, H, R), dtype=np.int32)
+    log_gate = np.full((B, H, R, K), NEG_INF)
+    lse_s = np.full((B, H, R), NEG_INF)
+    for b, (_, L) in enumerate(seq_bounds(cu_seqlens)):
+        nb = n_blocks(L)
+        if nb == 0:
+            continue
+        out = select(s[b:b + 1, :, :nb], K, prefill_history(nb))
+        idx[b, :, :nb], cnt[b, :, :nb], log_gate[b, :, :nb], lse_s[b, :, :nb] = (x[0] for x in out)
+    return idx, cnt, log_gate, lse_s
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, idx, cnt, log_gate, sm_scale, max_seqlen: int, seqs=None):
+    """attn_fwd() per sequence of a packed batch: q [T,Hq,D], k/v [T,Hkv,D].
+
+    Returns o fp64 [T,Hq,D] and lse fp64 [B,Hq,max_seqlen]; entries past a
+    sequence's length, and rows of sequences outside ``seqs``, are NaN.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    idx, cnt, log_gate = _i64(idx), _i64(cnt), _f64(log_gate)
+    bounds = seq_bounds(cu_seqlens)
+    o = np.full(q.shape, np.nan)
+    lse = np.full((len(bounds), q.shape[1], max_seqlen), np.nan)
+    for b, (st, L) in enumerate(bounds):
+        if L == 0 or (seqs is not None and b not in seqs):
+            continue
+        nb = n_blocks(L)
+        rows = slice(st, st + L)
+        ob, lb = attn_fwd(q[None, rows], k[None, rows], v[None, rows], idx[b:b + 1, :, :nb],
+                          cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], sm_scale)
+        o[rows] = ob[0]
+        lse[b, :, :L] = lb[0]
+    return o, lse
+
+
+def attn_bwd_varlen(q, k, v, do, cu_seqlens, idx, cnt, log_gate, s, sm_scale, seqs=None):
+    """attn_bwd() per sequence of a packed batch. Returns dq, dk, dv ([T, H, D])
+    and ds [B, Hkv, R, ld] (padding rows and sequences outside ``seqs`` zero)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    idx, cnt, log_gate, s = _i64(idx), _i64(cnt), _f64(log_gate), _f64(s)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    ds = np.zeros(s.shape)
+    for b, (st, L) in enumerate(seq_bounds(cu_seqlens)):
+        if L == 0 or (seqs is not None and b not in seqs):
+            continue
+        nb = n_blocks(L)
+        rows = slice(st, st + L)
+        g = attn_bwd(q[None, rows], k[None, rows], v[None, rows], do[None, rows], idx[b:b + 1, :, :nb],
+                     cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], s[b:b + 1, :, :nb, :nb], sm_scale)
+        dq[rows], dk[rows], dv[rows] = g[0][0], g[1][0], g[2][0]
+        ds[b, :, :nb, :nb] = g[3][0]
+    return dq, dk, dv, ds
 
 
 # ----------------------------------------------------------------------------

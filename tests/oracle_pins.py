@@ -16,7 +16,8 @@ Sources of truth used here:
 * brute force with Python loops on tiny inputs,
 * central finite differences in fp64,
 * invariants: shift invariance in s, exact zero influence of unselected K/V,
-  rows of ds sum to zero, probabilities sum to one.
+  rows of ds sum to zero, probabilities sum to one, causality (a sequence
+  cut inside a block gives the first rows of the longer sequence).
 """
 from __future__ import annotations
 
@@ -470,8 +471,147 @@ def pin_standin_scores(O):
     assert np.all(s1[:, 0] == 0.0) and np.any(s1[:, 1] != 0.0)
 
 
+def _sas_bias(s_rows, L, K):
+    """Additive mask of one sequence of L tokens (last block possibly partial) from
+    the rank selection and scipy gates: [L, L]."""
+    NQB = (L + BLOCK - 1) // BLOCK
+    bias = np.full((L, L), -np.inf)
+    for i in range(NQB):
+        row = np.asarray(s_rows[i, :i], dtype=np.float64)
+        ls = sp_logsumexp(row) if i else 0.0
+        r0, r1 = i * BLOCK, min(L, (i + 1) * BLOCK)
+        for j in _rank_select(list(row), K):
+            bias[r0:r1, j * BLOCK:(j + 1) * BLOCK] = row[j] - ls
+        for r in range(r0, r1):
+            bias[r, r0:r + 1] = 0.0
+    return bias
+
+
+def pin_partial_block_sdpa(O):
+    """A length that is not a multiple of 64: SDPA with the rank-selection mask."""
+    S, Hq, Hkv, D, K = 229, 4, 2, 8, 2
+    G = Hq // Hkv
+    q, k, v = _rand((1, S, Hq, D), 121), _rand((1, S, Hkv, D), 122), _rand((1, S, Hkv, D), 123)
+    NQB = 4
+    s = _rand((1, Hkv, NQB, NQB), 124, 1.5).astype(np.float32)
+    idx, cnt, lg, _ = O.select(s, K, O.prefill_history(NQB))
+    sc = 1.0 / math.sqrt(D)
+    o, lse = O.attn_fwd(q, k, v, idx, cnt, lg, sc)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    for h in range(Hkv):
+        bias = _sas_bias(s[0, h], S, K)
+        for g in range(G):
+            hq = h * G + g
+            ref = _sdpa(q[0, :, hq], k[0, :, h], v[0, :, h], bias, sc)
+            assert np.allclose(o[0, :, hq], ref, rtol=1e-12, atol=1e-12)
+            ref_lse = torch.logsumexp(torch.from_numpy(sc * q[0, :, hq] @ k[0, :, h].T + bias), dim=1).numpy()
+            assert np.allclose(lse[0, hq], ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def pin_partial_block_prefix(O):
+    """Causality: a sequence cut at S = 229 gives the first 229 rows of the same
+    sequence at 256 (its last block full), forward and backward, when the longer
+    sequence's extra rows carry no upstream gradient; the extra keys get none."""
+    S, S2, Hq, Hkv, D, K = 229, 256, 4, 2, 8, 2
+    q, k, v = _rand((1, S2, Hq, D), 131), _rand((1, S2, Hkv, D), 132), _rand((1, S2, Hkv, D), 133)
+    do = _rand((1, S2, Hq, D), 134)
+    do[:, S:] = 0.0
+    s = _rand((1, Hkv, 4, 4), 135)
+    sel = O.select(s, K, O.prefill_history(4))
+    sc = 0.37
+    o1, l1 = O.attn_fwd(q[:, :S], k[:, :S], v[:, :S], *sel[:3], sc)
+    o2, l2 = O.attn_fwd(q, k, v, *sel[:3], sc)
+    assert np.allclose(o1, o2[:, :S], rtol=0, atol=1e-13) and np.allclose(l1, l2[:, :, :S], rtol=0, atol=1e-13)
+    g1 = O.attn_bwd(q[:, :S], k[:, :S], v[:, :S], do[:, :S], *sel[:3], s, sc)
+    g2 = O.attn_bwd(q, k, v, do, *sel[:3], s, sc)
+    for a, b in zip(g1[:3], g2[:3]):
+        assert np.allclose(a, b[:, :S], rtol=0, atol=1e-12)
+    assert np.all(g2[1][:, S:] == 0.0) and np.all(g2[2][:, S:] == 0.0)
+    assert np.allclose(g1[3], g2[3], rtol=0, atol=1e-12)
+    assert np.abs(g1[3]).max() > 1e-3       # the gate gradients are exercised
+
+
+def _varlen_case(seed):
+    lens = [100, 64, 1, 229, 0, 130]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T, Hq, Hkv, D = int(cu[-1]), 4, 2, 8
+    q, k, v = _rand((T, Hq, D), seed), _rand((T, Hkv, D), seed + 1), _rand((T, Hkv, D), seed + 2)
+    R = 4
+    s = _rand((len(lens), Hkv, R, R), seed + 3).astype(np.float32)
+    return lens, cu, q, k, v, s
+
+
+def pin_varlen_sdpa(O):
+    """A packed batch of sequences of lengths 100, 64, 1, 229, 0, 130 against SDPA over
+    all packed rows with a mask that is each sequence's SAS mask on its diagonal block
+    and -inf between sequences; padding rows of the selection are empty."""
+    lens, cu, q, k, v, s = _varlen_case(141)
+    K, Hq, Hkv, D = 2, 4, 2, 8
+    G = Hq // Hkv
+    T = int(cu[-1])
+    idx, cnt, lg, lse_s = O.select_varlen(s, K, cu)
+    for b, L in enumerate(lens):
+        nb = (L + BLOCK - 1) // BLOCK
+        assert np.all(cnt[b, :, nb:] == 0) and np.all(idx[b, :, nb:] == -1) and np.all(np.isneginf(lse_s[b, :, nb:]))
+    sc = 1.0 / math.sqrt(D)
+    o, lse = O.attn_fwd_varlen(q, k, v, cu, idx, cnt, lg, sc, max(lens))
+    for h in range(Hkv):
+        bias = np.full((T, T), -np.inf)
+        for b, L in enumerate(lens):
+            if L:
+                st = int(cu[b])
+                bias[st:st + L, st:st + L] = _sas_bias(s[b, h], L, K)
+        for g in range(G):
+            hq = h * G + g
+            ref = _sdpa(q[:, hq], k[:, h], v[:, h], bias, sc)
+            assert np.allclose(o[:, hq], ref, rtol=1e-12, atol=1e-12)
+            ref_lse = torch.logsumexp(torch.from_numpy(sc * q[:, hq] @ k[:, h].T + bias), dim=1).numpy()
+            for b, L in enumerate(lens):
+                st = int(cu[b])
+                assert np.allclose(lse[b, hq, :L], ref_lse[st:st + L], rtol=1e-12, atol=1e-12)
+                assert np.all(np.isnan(lse[b, hq, L:]))
+
+
+def pin_varlen_finite_differences(O):
+    """Gradients of the packed batch against central finite differences of its loss."""
+    lens, cu, q, k, v, s = _varlen_case(151)
+    K, sc, h = 2, 0.3, 1e-6
+    do = _rand(q.shape, 155)
+    idx, cnt, lg, _ = O.select_varlen(s, K, cu)
+    dq, dk, dv, ds = O.attn_bwd_varlen(q, k, v, do, cu, idx, cnt, lg, s, sc)
+
+    def loss(q, k, v, s):
+        sel = O.select_varlen(s, K, cu)
+        o, _ = O.attn_fwd_varlen(q, k, v, cu, *sel[:3], sc, max(lens))
+        return float(np.sum(o * do))
+
+    r = np.random.default_rng(156)
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for _ in range(8):
+            pos = tuple(int(r.integers(0, n)) for n in grad.shape)
+            args = dict(q=q, k=k, v=v)
+            plus, minus = args[name].copy(), args[name].copy()
+            plus[pos] += h
+            minus[pos] -= h
+            lp = loss(**{**args, name: plus}, s=s)
+            lm = loss(**{**args, name: minus}, s=s)
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[pos]) <= 1e-6 * max(1.0, abs(fd)), (name, pos, fd, grad[pos])
+    for b, i, j in ((0, 1, 0), (3, 3, 1), (3, 2, 0), (5, 2, 1)):
+        plus, minus = s.copy(), s.copy()
+        plus[b, 1, i, j] += np.float32(1e-3)
+        minus[b, 1, i, j] -= np.float32(1e-3)
+        step = float(plus[b, 1, i, j]) - float(minus[b, 1, i, j])
+        fd = (loss(q, k, v, plus) - loss(q, k, v, minus)) / step
+        assert abs(fd - ds[b, 1, i, j]) <= 1e-5 * max(1.0, abs(fd)), (b, i, j, fd, ds[b, 1, i, j])
+    for b, L in enumerate(lens):
+        nb = (L + BLOCK - 1) // BLOCK
+        assert np.all(ds[b, :, nb:] == 0.0)
+
+
 ALL_PINS = [
     pin_topk_rank, pin_select_gates, pin_golden, pin_dense_equivalence, pin_block_diagonal,
     pin_general_sdpa, pin_bruteforce_loops, pin_finite_differences, pin_shift_invariance,
     pin_sparsity, pin_probabilities, pin_decode_vs_sdpa, pin_decode_vs_prefill, pin_standin_scores,
+    pin_partial_block_sdpa, pin_partial_block_prefix, pin_varlen_sdpa, pin_varlen_finite_differences,
 ]

@@ -26,15 +26,16 @@ MUTANTS = {
     "gate_sign_flipped": ("log_gate[b, h, r, slot] = row[j] - lse", "log_gate[b, h, r, slot] = lse - row[j]"),
     "tie_break_higher_index": ("np.lexsort((np.arange(nh), -s_row))", "np.lexsort((-np.arange(nh), -s_row))"),
     "causal_mask_off_by_one": ("np.where(u <= t, 0.0, NEG_INF)", "np.where(u < t + (t == 0), 0.0, NEG_INF)"),
-    "current_block_gated": ("bias[:, i * BLOCK:(i + 1) * BLOCK] = np.where(u <= t, 0.0, NEG_INF)",
-                            "bias[:, i * BLOCK:(i + 1) * BLOCK] = np.where(u <= t, (gates[0] if gates else 0.0), NEG_INF)"),
+    "current_block_gated": ("bias[:, rows] = np.where(u <= t, 0.0, NEG_INF)",
+                            "bias[:, rows] = np.where(u <= t, (gates[0] if gates else 0.0), NEG_INF)"),
     "scale_applied_to_gate": ("L = sm_scale * (Qi @ Kh.T) + stripe_bias(i, S, sel, gates)",
                               "L = sm_scale * ((Qi @ Kh.T) + stripe_bias(i, S, sel, gates))"),
     "gqa_head_map_modulo": ("h = hq // G\n    sel, gates", "h = hq % k.shape[2]\n    sel, gates"),
     "jacobian_term_dropped": ("ds[b, h, i, :i] = -p * tot", "ds[b, h, i, :i] = 0.0 * p * tot"),
     "dk_missing_scale": ("dk[b, :, h, :] += sm_scale * (dS.T @ Qi)", "dk[b, :, h, :] += (dS.T @ Qi)"),
     "dP_wrong_operand": ("dP = dOi @ Vh.T", "dP = dOi @ Kh.T"),
-    "gate_sum_wrong_axis": ("reshape(BLOCK, i, BLOCK).sum(axis=(0, 2))", "reshape(BLOCK, i, BLOCK).sum(axis=(2, 0))[::-1]"),
+    "gate_sum_wrong_axis": ("reshape(len(Qi), i, BLOCK).sum(axis=(0, 2))",
+                            "reshape(len(Qi), i, BLOCK).sum(axis=(2, 0))[::-1]"),
     "Dr_dropped": ("dS = P * (dP - Dr)", "dS = P * dP"),
     "decode_current_block_short": ("bias[c * BLOCK:L] = 0.0", "bias[c * BLOCK:L - 1 + (L - 1 == c * BLOCK)] = 0.0"),
     "decode_history_includes_current": ("return (_i64(kv_len) - 1) // BLOCK", "return (_i64(kv_len) + BLOCK - 1) // BLOCK"),
@@ -58,6 +59,18 @@ MUTANTS = {
                                   "qp = q.reshape(B, NQB, BLOCK, G, Hkv, D).mean(axis=(2, 3))"),
     "standin_scale_d": ("s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)",
                         "s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / D"),
+    "partial_block_keys_dropped": ("bias[:, rows] = np.where(u <= t, 0.0, NEG_INF)",
+                                   "bias[:, rows.start:rows.start + n - (n < BLOCK)] = np.where(u <= t, 0.0, NEG_INF)[:, :n - (n < BLOCK)]"),
+    "varlen_kv_of_first_sequence": ("ob, lb = attn_fwd(q[None, rows], k[None, rows], v[None, rows],",
+                                    "ob, lb = attn_fwd(q[None, rows], k[None, :L], v[None, :L],"),
+    "varlen_selection_of_first_sequence": ("        ob, lb = attn_fwd(q[None, rows], k[None, rows], v[None, rows], idx[b:b + 1, :, :nb],\n"
+                                           "                          cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], sm_scale)",
+                                           "        ob, lb = attn_fwd(q[None, rows], k[None, rows], v[None, rows], idx[:1, :, :nb],\n"
+                                           "                          cnt[:1, :, :nb], log_gate[:1, :, :nb], sm_scale)"),
+    "varlen_bwd_dk_misplaced": ("dq[rows], dk[rows], dv[rows] = g[0][0], g[1][0], g[2][0]",
+                                "dq[rows], dk[rows], dv[rows] = g[0][0], g[2][0], g[1][0]"),
+    "varlen_ds_scores_of_first_sequence": ("cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], s[b:b + 1, :, :nb, :nb], sm_scale)",
+                                           "cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], s[:1, :, :nb, :nb], sm_scale)"),
     "standin_transposed": ("s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)",
                            "s[b, h] = (kp[b, :, h, :] @ qp[b, :, h, :].T) / math.sqrt(D)"),
 }

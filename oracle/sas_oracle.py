@@ -419,6 +419,27 @@ def standin_scores(q, k, noise):
     return s + noise
 
 
+def standin_scores_decode(q, k_cache, page_table, kv_len, noise):
+    """Stand-in scores of decode queries: s[n, h, j] = mean over the G query heads of KV
+    head h of q[n] . mean over the 64 rows of page page_table[n, j] of k_cache[:, h] /
+    sqrt(D) + noise[n, h, j], in fp64, for the history blocks j < (kv_len[n]-1)//64 (the
+    other entries are NaN). q [N,Hq,D], k_cache [P,Hkv,64,D], noise [N,Hkv,ld]."""
+    q, kc, noise = _f64(q), _f64(k_cache), _f64(noise)
+    pt, kv_len = _i64(page_table), _i64(kv_len)
+    N, Hq, D = q.shape
+    Hkv = kc.shape[1]
+    G = Hq // Hkv
+    s = np.full(noise.shape, np.nan)
+    for n in range(N):
+        nh = int((kv_len[n] - 1) // BLOCK)
+        for h in range(Hkv):
+            qm = q[n, h * G:(h + 1) * G].mean(axis=0)
+            for j in range(nh):
+                km = kc[pt[n, j], h].mean(axis=0)
+                s[n, h, j] = float(qm @ km) / math.sqrt(D) + noise[n, h, j]
+    return s
+
+
 # ----------------------------------------------------------------------------
 # Work counts used to express throughput (not part of the method).
 # ----------------------------------------------------------------------------

@@ -609,9 +609,57 @@ def pin_varlen_finite_differences(O):
         assert np.all(ds[b, :, nb:] == 0.0)
 
 
+def pin_standin_scores_decode(O):
+    """Decode stand-in scores against explicit loops, the prefill stand-in, a closed form
+    and invariance to where the pages sit in the cache."""
+    N, Hq, Hkv, D = 3, 6, 2, 8
+    G = Hq // Hkv
+    lens = [1, 130, 200]
+    maxp = 4
+    P = 12
+    q = _rand((N, Hq, D), 161)
+    kc = _rand((P, Hkv, BLOCK, D), 162)
+    pt = np.array([[5, 0, 0, 0], [7, 2, 9, 0], [1, 11, 3, 4]])
+    noise = _rand((N, Hkv, maxp), 163)
+    s = O.standin_scores_decode(q, kc, pt, np.array(lens), noise)
+    for n, L in enumerate(lens):
+        nh = (L - 1) // BLOCK
+        assert np.all(np.isnan(s[n, :, nh:]))
+        for h in range(Hkv):
+            for j in range(nh):
+                dot = 0.0
+                for d in range(D):
+                    qm = sum(q[n, h * G + g, d] for g in range(G)) / G
+                    km = sum(kc[pt[n, j], h, t, d] for t in range(BLOCK)) / BLOCK
+                    dot += qm * km
+                assert abs(s[n, h, j] - (dot / math.sqrt(D) + noise[n, h, j])) < 1e-12
+    # a prefill query block whose 64 rows are one token repeated scores history blocks
+    # like that token's decode query
+    S = 3 * BLOCK
+    kp = _rand((1, S, Hkv, D), 164)
+    qp = np.repeat(q[2][None, None], BLOCK, axis=1)                   # [1, 64, Hq, D]
+    qfull = np.concatenate([np.zeros((1, 2 * BLOCK, Hq, D)), qp], axis=1)
+    sp = O.standin_scores(qfull, kp, np.zeros((1, Hkv, 3, 3)))
+    kc2 = kp[0].reshape(3, BLOCK, Hkv, D).transpose(0, 2, 1, 3)       # pages 0, 1, 2 in order
+    sd = O.standin_scores_decode(q[2:3], kc2, np.array([[0, 1, 2]]), np.array([2 * BLOCK + 1]),
+                                 np.zeros((1, Hkv, 3)))
+    assert np.allclose(sd[0, :, :2], sp[0, :, 2, :2], rtol=0, atol=1e-12)
+    # closed form: constant q = a, k = c gives a * c * sqrt(D)
+    c = O.standin_scores_decode(np.full((1, 4, 16), 0.5), np.full((2, 2, BLOCK, 16), -2.0), np.array([[1, 0]]),
+                                np.array([129]), np.zeros((1, 2, 2)))
+    assert np.allclose(c, 0.5 * -2.0 * 4.0, rtol=1e-14)
+    # moving the pages elsewhere in the cache (and the table with them) changes nothing
+    perm = np.random.default_rng(165).permutation(P)
+    inv = np.argsort(perm)
+    s2 = O.standin_scores_decode(q, kc[perm], inv[pt], np.array(lens), noise)
+    assert np.array_equal(np.isnan(s), np.isnan(s2)) and np.allclose(s[~np.isnan(s)], s2[~np.isnan(s2)], rtol=0,
+                                                                      atol=1e-13)
+
+
 ALL_PINS = [
     pin_topk_rank, pin_select_gates, pin_golden, pin_dense_equivalence, pin_block_diagonal,
     pin_general_sdpa, pin_bruteforce_loops, pin_finite_differences, pin_shift_invariance,
     pin_sparsity, pin_probabilities, pin_decode_vs_sdpa, pin_decode_vs_prefill, pin_standin_scores,
     pin_partial_block_sdpa, pin_partial_block_prefix, pin_varlen_sdpa, pin_varlen_finite_differences,
+    pin_standin_scores_decode,
 ]

@@ -71,6 +71,10 @@ MUTANTS = {
                                 "dq[rows], dk[rows], dv[rows] = g[0][0], g[2][0], g[1][0]"),
     "varlen_ds_scores_of_first_sequence": ("cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], s[b:b + 1, :, :nb, :nb], sm_scale)",
                                            "cnt[b:b + 1, :, :nb], log_gate[b:b + 1, :, :nb], s[:1, :, :nb, :nb], sm_scale)"),
+    "standin_decode_page_not_gathered": ("km = kc[pt[n, j], h].mean(axis=0)", "km = kc[j, h].mean(axis=0)"),
+    "standin_decode_query_head_zero": ("qm = q[n, h * G:(h + 1) * G].mean(axis=0)", "qm = q[n, h * G]"),
+    "standin_decode_history_includes_current": ("nh = int((kv_len[n] - 1) // BLOCK)\n        for h in range(Hkv):\n            qm",
+                                                "nh = int((kv_len[n] + BLOCK - 1) // BLOCK)\n        for h in range(Hkv):\n            qm"),
     "standin_transposed": ("s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)",
                            "s[b, h] = (kp[b, :, h, :] @ qp[b, :, h, :].T) / math.sqrt(D)"),
 }

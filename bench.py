@@ -15,12 +15,23 @@ Multi-GPU (torchrun): every rank runs its own independent replica of the
 workload (different seed), no collective in the data path; the timed region
 is bracketed by barriers and the max over ranks is reported (weak scaling).
 
+Beside that headline line, after the timed steps (rank 0 prints them as extra
+keys of the same JSON line): the Qwen3-4B 8k and Qwen3-14B 2x32k layers
+(`configs`), the full-history variant (K >= #history) of the 32k layer with
+its dk/dv load balance (`full_history`), the fused stand-in scorer + select
+(`score_select`), and a decode scaling study over 64K-512K of context at batch
+1 and 8, sparse against the same kernel reading every block (`decode_scaling`,
+CUDA-graph replays). Every extra number is the median of CUDA-event times of
+back-to-back CUDA-graph replays (so short calls carry no host launch gaps; a
+small call's inputs may then sit in L2).
+
 `--impl reference` times the fp64 CPU oracle instead (rank 0 only), each
 step a bounded sample of the same workload.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -47,6 +58,7 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--no-extras", action="store_true", help="skip the extra configs and studies")
     return ap.parse_args()
 
 
@@ -122,17 +134,35 @@ def select_bytes(nh_total, rows, K):
 
 
 # ---------------------------------------------------------------------------
-# DRAM bytes (read + write) per call of each entry point, summed over its kernels,
-# from one `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` capture of
-# run_once on the workload (profiles/dram_traffic_qwen3-8b-32k.md); to be
-# retaken whenever one of those kernels changes.
+# DRAM bytes (read + write) per call of each entry point, summed over its
+# kernels, from one `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum`
+# capture of run_once on the workload. Each figure carries the hash of the
+# kernel sources it was taken on; when the sources change the figure is no
+# longer reported (traffic: null) until it is captured again.
 # ---------------------------------------------------------------------------
-DRAM_TRAFFIC = {
-    "qwen3-8b-32k": {
-        "sas_attn_fwd": 405804800 + 236452864,
-        "sas_attn_bwd": (684000768 + 238927872) + (4346328320 + 128374016) + (536907008 + 3521024),
-    },
+TRAFFIC_SOURCES = {
+    "sas_attn_fwd": ["attn_fwd_sm100.cu", "sm100.cuh", "common.cuh"],
+    "sas_attn_bwd": ["attn_bwd_sm100.cu", "attn_simt.cu", "sm100.cuh", "common.cuh"],
 }
+DRAM_TRAFFIC = {
+    # workload -> entry point -> (bytes per call, sha256[:16] of the sources above)
+}
+
+
+def sources_hash(entry):
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES[entry]:
+        with open(os.path.join(HERE, "trainable_gated_block_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, entry):
+    """DRAM bytes per call recorded for the current kernel sources, else None."""
+    rec = DRAM_TRAFFIC.get(workload, {}).get(entry)
+    if rec is None or entry not in TRAFFIC_SOURCES or rec[1] != sources_hash(entry):
+        return None
+    return rec[0]
 
 
 # ---------------------------------------------------------------------------
@@ -265,7 +295,7 @@ def run_ours(a):
         dist.barrier()
     sas.get_error_flag()
     total_ms = t0.elapsed_time(t1)
-    part_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / a.steps for i, n in enumerate(names)}
+    part_ms = {n: statistics.median(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
     prefill_ms = part_ms["select"] + part_ms["fwd"] + part_ms["bwd"]
     dec_ms = part_ms["dselect"] + part_ms["decode"]
     t = max_over_ranks([total_ms, prefill_ms, dec_ms] + [part_ms[n] for n in names], dist, dev)
@@ -303,7 +333,7 @@ def run_ours(a):
     }
     dom = max(("fwd", "bwd", "decode", "select"), key=lambda n: part_ms[n])
     kd = kernels[dom]
-    traffic = DRAM_TRAFFIC.get(pc.name, {}).get(f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}")
+    traffic = recorded_traffic(pc.name, f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}")
     roofline = dict(bound=kd["bound"], achieved=round(kd["achieved"], 3), peak=kd["peak"], unit=kd["unit"],
                     frac=round(kd["frac"], 4), traffic=traffic, kernel=f"sas_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom}",
                     peak_note=f"{tag} ({tnote if kd['bound'] == 'tensor' else 'HBM copy'})")
@@ -311,6 +341,9 @@ def run_ours(a):
     e2e = None
     if not a.no_e2e:
         e2e = run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, world, dist, dev)
+    extras = {}
+    if rank == 0 and not a.no_extras:
+        extras = run_extras(torch, sas, inputs, P, px, pc, dev, peaks, tpeak, a)
 
     line = None
     if rank == 0:
@@ -339,13 +372,220 @@ def run_ours(a):
             "gpu_launches": launches,
             "e2e": e2e,
         }
+        line.update(extras)
         if world == 1 and not a.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(pc, px, a.cpu_seconds)
+            if not a.no_extras:
+                # the oracle on the other two prefill workloads (fewer stripes each)
+                per = {pc.name: dict(tflops=line["cpu_baseline"]["value"],
+                                     parts_s=line["cpu_baseline"]["parts_s"])}
+                for name in ("qwen3-4b-8k", "qwen3-14b-2x32k"):
+                    cfg = inputs.workload(name)
+                    cb = cpu_baseline(cfg, inputs.make_prefill(cfg), a.cpu_seconds / 3)
+                    per[name] = dict(tflops=cb["value"], parts_s=cb["parts_s"], sample=cb["sample"])
+                line["cpu_baseline"]["per_config"] = per
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if line is not None:
         print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# extra measurements (rank 0, after the timed steps)
+# ---------------------------------------------------------------------------
+
+def _graph(torch, fns):
+    """Capture the callables (run once eagerly first) into one CUDA graph."""
+    for fn in fns:
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        for fn in fns:
+            fn()
+    return g
+
+
+def _replay_ms(torch, g, reps=20, warmup=3):
+    """Median device time (ms) of back-to-back replays of graph g (no host gap between
+    them, so short calls are not padded by launch overhead)."""
+    for _ in range(warmup):
+        g.replay()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record()
+    for k in range(reps):
+        g.replay()
+        ev[k + 1].record()
+    torch.cuda.synchronize()
+    return statistics.median(ev[k].elapsed_time(ev[k + 1]) for k in range(reps))
+
+
+def _prefill_parts(torch, sas, P, cfg, K, ws, reps, warmup):
+    """Median replay time of select, forward and backward, each captured in its own graph."""
+    sc = 1.0 / math.sqrt(cfg.D)
+    st = {}
+
+    def sel():
+        st["sel"] = sas.select(P["s"], K)
+
+    def fwd():
+        st["o"] = sas.attn_fwd(P["q"], P["k"], P["v"], *st["sel"][:3], sc)
+
+    def bwd():
+        sl = st["sel"]
+        sas.attn_bwd(P["q"], P["k"], P["v"], st["o"][0], P["do"], st["o"][1], P["s"], sl[3], sl[0], sl[1], sl[2], sc,
+                     workspace=ws)
+
+    graphs = [(n, _graph(torch, [fn])) for n, fn in (("select", sel), ("fwd", fwd), ("bwd", bwd))]
+    ms = {n: _replay_ms(torch, g, reps, warmup) for n, g in graphs}
+    del graphs
+    return ms, st
+
+
+def _prefill_line(cfg, K, ms, tpeak, hbm):
+    tiles = sum(min(K, i) + 1 for i in range(cfg.NQB)) * cfg.B * cfg.Hq
+    unit = 64 * 64 * cfg.D
+    pre = ms["select"] + ms["fwd"] + ms["bwd"]
+    tf = lambda f, t: f * unit * tiles / (t * 1e-3) / 1e12          # noqa: E731
+    return dict(B=cfg.B, S=cfg.S, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D, K=K, attended_tiles=tiles,
+                ms={k: round(v, 4) for k, v in ms.items()},
+                tflops_prefill=round(tf(14, pre), 2), frac_prefill=round(tf(14, pre) / tpeak, 4),
+                tflops_fwd=round(tf(4, ms["fwd"]), 2), frac_fwd=round(tf(4, ms["fwd"]) / tpeak, 4),
+                tflops_bwd=round(tf(10, ms["bwd"]), 2), frac_bwd=round(tf(10, ms["bwd"]) / tpeak, 4))
+
+
+def _dkv_balance(idx, NQB, n_bh, ctas):
+    """Steps per CTA of the dk/dv kernel's deal, modelled on the host from the selection
+    (items = key blocks; a key block's steps = its own block + every query block that kept
+    it; longest first within a head, dealt in snake order over the CTAs): max / mean."""
+    import numpy as np
+    steps = np.ones((n_bh, NQB), dtype=np.int64)                  # own block
+    for bh in range(n_bh):
+        sel = idx[bh][idx[bh] >= 0]
+        steps[bh] += np.bincount(sel.ravel(), minlength=NQB)[:NQB]
+    order = [(bh, int(j)) for bh in range(n_bh) for j in np.argsort(-steps[bh], kind="stable")]
+    per = np.zeros(ctas, dtype=np.int64)
+    for pos, (bh, j) in enumerate(order):
+        r, c = divmod(pos, ctas)
+        per[c if r % 2 == 0 else ctas - 1 - c] += steps[bh, j]
+    return dict(items=len(order), steps_max_item=int(steps.max()), steps_mean_item=round(float(steps.mean()), 2),
+                cta_steps_max=int(per.max()), cta_steps_mean=round(float(per.mean()), 2),
+                cta_max_over_mean=round(float(per.max() / per.mean()), 4))
+
+
+def run_extras(torch, sas, inputs, P, px, pc, dev, peaks, tpeak, a):
+    out = {}
+    warmup = 2
+    # --- the other two prefill workloads
+    cfgs = {}
+    for name in ("qwen3-4b-8k", "qwen3-14b-2x32k"):
+        cfg = inputs.workload(name)
+        x = {k: v.to(dev) for k, v in inputs.make_prefill(cfg).items()}
+        ws = torch.empty(sas.bwd_workspace_bytes(x["q"], x["k"], cfg.K), dtype=torch.uint8, device=dev)
+        ms, _ = _prefill_parts(torch, sas, x, cfg, cfg.K, ws, 10, warmup)
+        cfgs[name] = _prefill_line(cfg, cfg.K, ms, tpeak, peaks["hbm"])
+        del x, ws
+        torch.cuda.empty_cache()
+    out["configs"] = cfgs
+    # --- the full-history variant on the headline workload's tensors
+    Kf = pc.NQB
+    ws = torch.empty(sas.bwd_workspace_bytes(P["q"], P["k"], Kf), dtype=torch.uint8, device=dev)
+    ms, st = _prefill_parts(torch, sas, P, pc, Kf, ws, 3, 1)
+    fh = _prefill_line(pc, Kf, ms, tpeak, peaks["hbm"])
+    import numpy as np
+    idx = st["sel"][0].cpu().numpy().reshape(pc.B * pc.Hkv, pc.NQB, Kf)
+    fh["dkv_balance"] = _dkv_balance(idx, pc.NQB, pc.B * pc.Hkv,
+                                     torch.cuda.get_device_properties(dev).multi_processor_count)
+    out["full_history"] = {pc.name: fh}
+    del ws, st
+    torch.cuda.empty_cache()
+    # --- fused stand-in scorer + select on the headline workload (its scores are the stand-in)
+    if "noise" in px:
+        noise = px["noise"].to(dev)
+        s_buf = torch.zeros_like(P["s"])
+        wsc = torch.empty(max(256, int(sas.lib().sas_score_select_workspace_size(pc.B, pc.S, pc.Hq, pc.Hkv, pc.D))),
+                          dtype=torch.uint8, device=dev)
+        g = _graph(torch, [lambda: sas.score_select(P["q"], P["k"], pc.K, noise=noise, workspace=wsc, s_out=s_buf)])
+        ms = {"score_select": _replay_ms(torch, g, 20, 3)}
+        del g
+        rows = pc.B * pc.Hkv * pc.NQB
+        nbytes = (P["q"].numel() + P["k"].numel()) * 2 + noise.numel() // 2 * 4 + \
+            sum(range(pc.NQB)) * pc.B * pc.Hkv * 4 + rows * (pc.K * 8 + 8)
+        out["score_select"] = dict(workload=pc.name, us=round(ms["score_select"] * 1e3, 2), bytes=int(nbytes),
+                                   gbs=round(nbytes / (ms["score_select"] * 1e-3) / 1e9, 1),
+                                   frac_hbm=round(nbytes / (ms["score_select"] * 1e-3) / 1e9 / peaks["hbm"], 4),
+                                   note="pooling reads q and k once; scores written once (lower triangle)")
+        del s_buf, wsc, noise
+    torch.cuda.empty_cache()
+    # --- decode scaling study
+    out["decode_scaling"] = decode_scaling(torch, sas, inputs, dev, peaks)
+    return out
+
+
+def decode_scaling(torch, sas, inputs, dev, peaks):
+    """Sparse (select + decode, K = 32; and the same with the stand-in scores computed from
+    the pooled-key cache first, `scored`) against the same decode kernel reading every block
+    (K >= #history, selection given), at 64K-512K of context, batch 1 and 8. Each arm is
+    captured in a CUDA graph and replayed; the median replay time is reported."""
+    Hq, Hkv, D, K = 32, 8, 128, 32
+    rows = []
+    for batch in (1, 8):
+        for ctx in (65536, 131072, 262144, 524288):
+            x = inputs.make_decode_device(batch, ctx, Hq, Hkv, D, seed=ctx + batch, device=dev)
+            nh = ctx // BLOCK
+            ws_s = torch.empty(max(256, sas.decode_workspace_bytes(batch, Hq, Hkv, D, K)), dtype=torch.uint8,
+                               device=dev)
+            ws_d = torch.empty(max(256, sas.decode_workspace_bytes(batch, Hq, Hkv, D, nh)), dtype=torch.uint8,
+                               device=dev)
+            dense_idx = torch.arange(nh, dtype=torch.int32, device=dev).expand(batch, Hkv, nh).contiguous()
+            dense_cnt = torch.full((batch, Hkv), nh, dtype=torch.int32, device=dev)
+            dense_lg = torch.full((batch, Hkv, nh), -math.log(nh), dtype=torch.float32, device=dev)
+            kpool = sas.pool_pages(x["k_cache"])      # pooled-key cache, filled once per page (not timed)
+            st = {}
+
+            def scored_sel():
+                st["sel"] = sas.score_select_decode(x["q"], kpool, x["page_table"], x["kv_len"], K, nh)[1:]
+
+            def sparse_sel():
+                st["sel"] = sas.select(x["s"], K, kv_len=x["kv_len"])
+
+            def sparse_dec():
+                sas.decode_paged(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["kv_len"], *st["sel"][:3],
+                                 workspace=ws_s, with_lse=False)
+
+            def dense_dec():
+                sas.decode_paged(x["q"], x["k_cache"], x["v_cache"], x["page_table"], x["kv_len"], dense_idx,
+                                 dense_cnt, dense_lg, workspace=ws_d, with_lse=False)
+
+            res = {}
+            for arm, fns in (("sparse", [sparse_sel, sparse_dec]), ("scored", [scored_sel, sparse_dec]),
+                             ("dense", [dense_dec])):
+                g = _graph(torch, fns)
+                res[arm] = _replay_ms(torch, g, 10, 2)
+                del g
+            for arm, fn in (("sparse_select", sparse_sel), ("scored_select", scored_sel)):
+                g = _graph(torch, [fn])
+                res[arm] = _replay_ms(torch, g, 10, 2)
+                del g
+            sas.get_error_flag()
+            kv_sparse = batch * Hkv * (K * BLOCK + 1) * D * 2 * 2
+            kv_dense = batch * Hkv * (nh * BLOCK + 1) * D * 2 * 2
+            rows.append(dict(batch=batch, context=ctx, K=K,
+                             us_sparse=round(res["sparse"] * 1e3, 2), us_sparse_select=round(res["sparse_select"] * 1e3, 2),
+                             us_scored=round(res["scored"] * 1e3, 2),
+                             us_scored_select=round(res["scored_select"] * 1e3, 2),
+                             us_dense=round(res["dense"] * 1e3, 2), speedup=round(res["dense"] / res["sparse"], 2),
+                             speedup_scored=round(res["dense"] / res["scored"], 2),
+                             scoring_share=round(res["scored_select"] / res["scored"], 3),
+                             dense_gbs=round(kv_dense / (res["dense"] * 1e-3) / 1e9, 1),
+                             dense_frac_hbm=round(kv_dense / (res["dense"] * 1e-3) / 1e9 / peaks["hbm"], 4),
+                             sparse_kv_bytes=kv_sparse, dense_kv_bytes=kv_dense))
+            del x, ws_s, ws_d, dense_idx, dense_cnt, dense_lg, st, kpool
+            torch.cuda.empty_cache()
+    return dict(rows=rows, note="kernel-level time of one decode step (graph replay); the pages' 2.4x/4.6x/5.6x "
+                                "(batch 1, 64K/256K/512K) and ~13x (batch 8, 64K) are whole-model serving latencies "
+                                "on other hardware, quoted as context only")
 
 
 def run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, world, dist, dev):
@@ -393,8 +633,8 @@ def run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, wo
     evs = [step(True) for _ in range(a.steps)]
     torch.cuda.synchronize()
     sas.get_error_flag()
-    pre = sum(e[0].elapsed_time(e[1]) for e in evs) / a.steps
-    dec = sum(e[1].elapsed_time(e[2]) for e in evs) / a.steps
+    pre = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    dec = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
     pre, dec = max_over_ranks([pre, dec], dist, dev)
     d2h = sum(t.numel() * t.element_size() for t in outs.values())
     return dict(value=round(weak_tflops(world, flops_fb, pre), 3), unit="TFLOPS",

@@ -31,7 +31,19 @@
  *     they record the first problem in a per-device status word that
  *     sas_get_error_flag() reports and clears (SAS_ERR_INVALID_ARG for bad
  *     device-side data, SAS_ERR_TIMEOUT when a bounded wait gave up).
- *   - Scores must be finite; NaN rows have no defined Top-K.
+ *   - Scores must be finite. A selection row whose history holds a NaN or
+ *     +-inf score is flagged (SAS_ERR_INVALID_ARG from sas_get_error_flag)
+ *     and gets the empty selection (cnt 0, idx -1, log_gate -inf) with
+ *     lse_s = NaN; the other rows are unaffected.
+ *   - Prefill sequences may have any length: a length that is not a multiple
+ *     of 64 ends in a partial block, which is a query block like the others
+ *     and (having no later block) is never selected as history. Batches of
+ *     different lengths use the _varlen entry points: q/k/v packed along the
+ *     token axis, sequence b at token rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *     (device int32 [B + 1], non-decreasing, cu_seqlens[B] <= total_tokens,
+ *     each length <= max_seqlen; a sequence that breaks this is flagged and
+ *     treated as empty), per-block tensors padded to ceil(max_seqlen / 64)
+ *     rows per sequence and the row LSE to max_seqlen.
  *   - Tensor layouts are row-major with the last named dimension contiguous.
  *     GQA: query head hq reads KV head hq / (Hq / Hkv).
  *   - Logits are sm_scale * q.k + log g: sm_scale multiplies q.k only.
@@ -81,6 +93,8 @@ sas_status sas_get_error_flag(void *stream);
  *          Else decode: device int32 [B]; every row of batch entry b has
  *          nh = (kv_len[b] - 1) / block_size history blocks (kv_len[b] >= 1;
  *          nh > ld_s is flagged and clamped to ld_s).
+ *          Rows hold at most 16384 history blocks (1M tokens); longer rows
+ *          return SAS_ERR_UNSUPPORTED.
  * K        budget in blocks, K >= 0. A row keeps min(K, nh) blocks.
  * idx      device int32 [B, Hkv, n_rows, K]: kept block indices, ascending,
  *          padded with -1. Order of the Top-K: score descending, then block
@@ -96,17 +110,34 @@ sas_status sas_select(const float *s, int B, int Hkv, int n_rows, int ld_s,
                       void *stream);
 
 /*
+ * sas_select_varlen - sas_select (prefill) for a packed batch of sequences of
+ * different lengths (the same method applied to each sequence, SAS review
+ * §2.2, §2.4). cu_seqlens: device int32 [B + 1] (see the conventions above).
+ * Row (b, h, r) is query block r of sequence b when r < ceil(len_b / 64);
+ * later rows are padding: cnt 0, idx -1, log_gate -inf, lse_s -inf, and their
+ * scores are not read. n_rows >= ceil(max_seqlen / 64), ld_s >= n_rows.
+ */
+sas_status sas_select_varlen(const float *s, int B, int Hkv, int n_rows, int ld_s,
+                             const int32_t *cu_seqlens, int block_size, int K,
+                             int32_t *idx, int32_t *cnt, float *log_gate, float *lse_s,
+                             void *stream);
+
+/*
  * sas_attn_fwd - gated block-sparse causal attention, forward.
  * SAS review §2.3, eq. o_SAS, with the current block kept at gate 1 (§2.4)
  * under a causal mask, tiled over the kept key blocks only (§2.6).
  *
  * dtype    SAS_BF16 (tensor cores, fp32 accumulation) or SAS_F32 (fp32
- *          FMA throughout).
+ *          FMA throughout). bf16 with D = 128 runs on the tcgen05 tensor
+ *          cores; fp32, and bf16 with D = 64, run on the CUDA cores (an
+ *          untuned path: fp32 keeps full fp32 arithmetic, D = 64 is a
+ *          secondary head size).
  * q        device [B, S, Hq, D]; k, v device [B, S, Hkv, D]; all of dtype,
- *          16-byte aligned. S % 64 == 0, Hq % Hkv == 0, D in {64, 128}.
- * idx, cnt, log_gate   as written by sas_select with n_rows = S/64 and the
- *          same K; an index outside 0..i-1 for query block i is flagged and
- *          skipped.
+ *          16-byte aligned. S >= 1 (the last block may be partial),
+ *          Hq % Hkv == 0, D in {64, 128}.
+ * idx, cnt, log_gate   as written by sas_select with n_rows = ceil(S/64) and
+ *          the same K; an index outside 0..i-1 for query block i is flagged
+ *          and skipped.
  * o        device [B, S, Hq, D] of dtype (output).
  * lse      device fp32 [B, Hq, S] (output): natural-log LSE of each row's
  *          logits, kept for the backward.
@@ -116,9 +147,29 @@ sas_status sas_attn_fwd(sas_dtype dtype, const void *q, const void *k, const voi
                         const int32_t *idx, const int32_t *cnt, const float *log_gate,
                         float sm_scale, void *o, float *lse, void *stream);
 
+/*
+ * sas_attn_fwd_varlen - sas_attn_fwd for a packed batch of sequences of
+ * different lengths (the method applied to each sequence on its own).
+ * q        device [total_tokens, Hq, D]; k, v [total_tokens, Hkv, D].
+ * cu_seqlens, max_seqlen   see the conventions above.
+ * idx, cnt, log_gate   from sas_select_varlen with n_rows = ceil(max_seqlen/64).
+ * o        device [total_tokens, Hq, D]; rows of no sequence are not written.
+ * lse      device fp32 [B, Hq, max_seqlen]; entries past a sequence's length
+ *          are not written.
+ */
+sas_status sas_attn_fwd_varlen(sas_dtype dtype, const void *q, const void *k, const void *v,
+                               const int32_t *cu_seqlens, int B, int max_seqlen, int total_tokens,
+                               int Hq, int Hkv, int D, int block_size, int K,
+                               const int32_t *idx, const int32_t *cnt, const float *log_gate,
+                               float sm_scale, void *o, float *lse, void *stream);
+
 /* Bytes of device workspace sas_attn_bwd needs for these sizes (0 on a bad
  * argument). */
 size_t sas_attn_bwd_workspace_size(sas_dtype dtype, int B, int S, int Hq, int Hkv, int D, int K);
+
+/* Bytes of device workspace sas_attn_bwd_varlen needs (0 on a bad argument). */
+size_t sas_attn_bwd_varlen_workspace_size(sas_dtype dtype, int B, int max_seqlen, int total_tokens,
+                                          int Hq, int Hkv, int D, int K);
 
 /*
  * sas_attn_bwd - gradients of the forward with respect to q, k, v and s.
@@ -134,11 +185,14 @@ size_t sas_attn_bwd_workspace_size(sas_dtype dtype, int B, int S, int Hq, int Hk
  * s, ld_s  the scores given to sas_select; lse_s its output.
  * dq       device [B, S, Hq, D] of dtype (output).
  * dk, dv   device [B, S, Hkv, D] of dtype (output).
- * ds       device fp32 [B, Hkv, S/64, ld_s] (output; every entry of each
- *          row 0..ld_s-1 is written).
+ * ds       device fp32 [B, Hkv, ceil(S/64), ld_s] (output; every entry of
+ *          each row 0..ld_s-1 is written).
  * workspace device, ws_bytes >= sas_attn_bwd_workspace_size(...), 256-byte
  *          aligned; contents on entry do not matter.
- * Summation order inside dk/dv may vary between runs (fp32 atomics).
+ * The bf16 D = 128 path writes dq, dk and dv once each (deterministic); the
+ * CUDA-core path accumulates dk/dv with fp32 atomics, whose summation order
+ * may vary between runs. The bf16 D = 128 path handles at most 32767 query
+ * blocks per sequence (S <= 2,097,088; SAS_ERR_UNSUPPORTED beyond).
  */
 sas_status sas_attn_bwd(sas_dtype dtype, const void *q, const void *k, const void *v,
                         const void *o, const void *dout, const float *lse,
@@ -147,6 +201,89 @@ sas_status sas_attn_bwd(sas_dtype dtype, const void *q, const void *k, const voi
                         int B, int S, int Hq, int Hkv, int D, int block_size, int K,
                         float sm_scale, void *dq, void *dk, void *dv, float *ds,
                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * sas_attn_bwd_varlen - sas_attn_bwd for a packed batch (layouts as in
+ * sas_attn_fwd_varlen; s and ds [B, Hkv, ceil(max_seqlen/64), ld_s], whose
+ * padding rows of ds are written as zero). dk/dv rows of no sequence are not
+ * written.
+ */
+sas_status sas_attn_bwd_varlen(sas_dtype dtype, const void *q, const void *k, const void *v,
+                               const void *o, const void *dout, const float *lse,
+                               const float *s, int ld_s, const float *lse_s,
+                               const int32_t *idx, const int32_t *cnt, const float *log_gate,
+                               const int32_t *cu_seqlens, int B, int max_seqlen, int total_tokens,
+                               int Hq, int Hkv, int D, int block_size, int K, float sm_scale,
+                               void *dq, void *dk, void *dv, float *ds,
+                               void *workspace, size_t ws_bytes, void *stream);
+
+/* Bytes of device workspace sas_score_select needs (0 on a bad argument). */
+size_t sas_score_select_workspace_size(int B, int S, int Hq, int Hkv, int D);
+
+/*
+ * sas_score_select - block-pooled stand-in selector scores, fused with the
+ * Top-K selection and the log-gates of sas_select (prefill).
+ * SAS review §2.2: the selector scores each history block of a query block,
+ * s = R_theta(q, {K_Bm}), and the Top-K are kept; §2.4, eq. log g. The
+ * trained selector (AttnGate) is not part of this library; its stand-in is
+ *   s[b,h,i,j] = mean over the 64 rows of block i and the G query heads of
+ *                KV head h of q, dotted with the mean over the 64 rows of
+ *                block j of k[:, :, h], divided by sqrt(D), plus noise[b,h,i,j]
+ * for j < i (fp32 sums of the bf16 inputs).
+ *
+ * q, k     device bf16 [B, S, Hq, D], [B, S, Hkv, D]; S % 64 == 0, D in
+ *          {64, 128}, 16-byte aligned.
+ * noise    device fp32 [B, Hkv, S/64, ld_noise] added to the scores, or NULL.
+ * s        device fp32 [B, Hkv, S/64, ld_s] (output): entries j < i of row
+ *          (b, h, i) are written, the others are left as they are. These are
+ *          the scores the backward's Jacobian needs.
+ * idx, cnt, log_gate, lse_s   as sas_select writes them for these scores.
+ * workspace device, 256-byte aligned, ws_bytes >= sas_score_select_workspace_size
+ *          (it holds the pooled queries and keys).
+ */
+sas_status sas_score_select(const void *q, const void *k, const float *noise, int ld_noise,
+                            int B, int S, int Hq, int Hkv, int D, int block_size, int K,
+                            float *s, int ld_s, int32_t *idx, int32_t *cnt, float *log_gate,
+                            float *lse_s, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * sas_pool_pages - the pooled-key cache of a paged KV cache, for the decode
+ * stand-in scorer: kpool[p, h, :] = the mean of the 64 key rows of page p and
+ * KV head h (fp32 sums of the bf16 keys). The stand-in for the selector of
+ * SAS review §2.2 scores a history block by its mean key; a serving engine
+ * computes it once, when a page fills, instead of at every decode step.
+ *
+ * k_cache  device bf16 [num_pages, Hkv, 64, D], D in {64, 128}, 16-byte aligned.
+ * pages    device int32 [n_pages] page ids to pool, or NULL for all pages.
+ *          An id outside [0, num_pages) is flagged and skipped.
+ * kpool    device fp32 [num_pages, Hkv, D] (output; only the listed pages are
+ *          written), 16-byte aligned.
+ */
+sas_status sas_pool_pages(const void *k_cache, int num_pages, int Hkv, int D, int page_size,
+                          const int32_t *pages, int n_pages, float *kpool, void *stream);
+
+/*
+ * sas_score_select_decode - decode stand-in scores from the pooled-key cache,
+ * then the decode selection (SAS review §2.2, §2.4). For sequence n (query at
+ * kv_len[n]-1, history blocks j < (kv_len[n]-1)/64) and KV head h:
+ *   s[n, h, j] = mean over the G query heads of h of q[n] . kpool[page_table[n, j], h]
+ *                / sqrt(D) + noise[n, h, j]
+ * then idx, cnt, log_gate, lse_s exactly as sas_select in decode mode.
+ *
+ * q          device bf16 [N, Hq, D]; kpool from sas_pool_pages.
+ * page_table device int32 [N, max_pages]; a bad page id is flagged and the
+ *            row gets a NaN score (so the selection flags it and keeps nothing).
+ * noise      device fp32 [N, Hkv, ld_noise] or NULL.
+ * s          device fp32 [N, Hkv, ld_s] (output; entries j < nh written),
+ *            ld_s >= the longest history (<= 16384 blocks).
+ * idx, cnt, log_gate, lse_s   device [N, Hkv, K], [N, Hkv], [N, Hkv, K], [N, Hkv].
+ */
+sas_status sas_score_select_decode(const void *q, const float *kpool, int num_pages,
+                                   const int32_t *page_table, int max_pages, const int32_t *kv_len,
+                                   int N, int Hq, int Hkv, int D, int page_size,
+                                   const float *noise, int ld_noise, int K, float *s, int ld_s,
+                                   int32_t *idx, int32_t *cnt, float *log_gate, float *lse_s,
+                                   void *stream);
 
 /* Bytes of device workspace sas_decode_paged needs (0 on a bad argument). */
 size_t sas_decode_workspace_size(int N, int Hq, int Hkv, int D, int K);
@@ -197,7 +334,10 @@ sas_status sas_decode_paged(const void *q, const void *k_cache, const void *v_ca
  * contents; nothing in it needs to start at zero. Calls that overlap on the
  * GPU (on different streams, or from threads without ordering) race on it.
  * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture.
+ * device current and caches it with the current context's id; the lookup is
+ * repeated when another context is current (after cudaDeviceReset). Make the
+ * first call on a device, and the first after a reset, before any stream
+ * capture.
  */
 sas_status sas_decode_paged_noalloc(const void *q, const void *k_cache, const void *v_cache,
                                     int num_pages, const int32_t *page_table, int max_pages,

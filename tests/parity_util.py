@@ -8,7 +8,8 @@ Tolerances (what the tests assert):
   magnitude >= 4 has a bf16 spacing of 2^-5, so rounding alone can move it
   by 2^-6 = 0.0156. There the test also requires the GPU value to be within
   1e-2 of the oracle value rounded to bf16 (RNE), and counts such elements.
-  lse max-abs <= 1e-2. Gradients dq, dk, dv, ds: relative L2 <= 1e-2.
+  lse max-abs <= 1e-2. Gradients dq, dk, dv, ds: relative L2 <= 1e-2; where the
+  exact gradient is identically zero, max-abs <= 1e-5 (rounding noise only).
 """
 from __future__ import annotations
 
@@ -18,6 +19,11 @@ import torch
 FP32_TOL = 1e-5
 BF16_OUT_TOL = 1e-2
 BF16_GRAD_REL_L2 = 1e-2
+
+# Every bf16 output comparison of the session: (what, elements, max_abs,
+# max_abs against the oracle rounded to bf16, elements that pass only through
+# the output-rounding exemption). Printed at the end of the run by conftest.py.
+OUT_LOG: list[tuple[str, int, float, float, int]] = []
 
 
 def np64(t):
@@ -62,8 +68,10 @@ def check_out(gpu, ref, dtype: str, what: str):
     bad = over & ~quant_only
     assert not np.any(bad), (f"{what}: bf16 max-abs {err.max():.3e} > {BF16_OUT_TOL} "
                              f"at {int(bad.sum())} elements not explained by output rounding")
-    return dict(max_abs=float(err.max(initial=0.0)), max_abs_vs_rounded=float(errq.max(initial=0.0)),
-                quantization_only=int(quant_only.sum()))
+    res = dict(max_abs=float(err.max(initial=0.0)), max_abs_vs_rounded=float(errq.max(initial=0.0)),
+               quantization_only=int(quant_only.sum()))
+    OUT_LOG.append((what, int(err.size), res["max_abs"], res["max_abs_vs_rounded"], res["quantization_only"]))
+    return res
 
 
 def check_grad(gpu, ref, dtype: str, what: str):
@@ -72,6 +80,13 @@ def check_grad(gpu, ref, dtype: str, what: str):
     if dtype == "f32":
         m = max_abs(g, r)
         assert m <= FP32_TOL, f"{what}: fp32 max-abs {m:.3e} > {FP32_TOL}"
+        return dict(max_abs=m)
+    if float(np.linalg.norm(r.ravel())) == 0.0:
+        # the exact gradient is zero (e.g. a lone token attending only itself: P = 1 and
+        # dP - Dr = 0): a relative error is undefined, so only rounding noise at the fp32
+        # level is allowed
+        m = float(np.abs(g).max(initial=0.0))
+        assert m <= FP32_TOL, f"{what}: exact gradient is zero, GPU max-abs {m:.3e} > {FP32_TOL}"
         return dict(max_abs=m)
     e = rel_l2(g, r)
     assert e <= BF16_GRAD_REL_L2, f"{what}: bf16 rel-L2 {e:.3e} > {BF16_GRAD_REL_L2}"

@@ -51,7 +51,7 @@ def _fwd(L, **kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(S=100), sas.SAS_ERR_INVALID_ARG),
+    (dict(S=0), sas.SAS_ERR_INVALID_ARG),
     (dict(Hq=3), sas.SAS_ERR_INVALID_ARG),
     (dict(K=-1), sas.SAS_ERR_INVALID_ARG),
     (dict(B=0), sas.SAS_ERR_INVALID_ARG),
@@ -70,13 +70,19 @@ def test_select_rejects_bad_arguments(L):
     assert f(None, 1, 1, 8, 8, None, 64, 2, FAKE, FAKE, FAKE, FAKE, None) == sas.SAS_ERR_INVALID_ARG
     assert f(FAKE, 1, 1, 8, 4, None, 64, 2, FAKE, FAKE, FAKE, FAKE, None) == sas.SAS_ERR_INVALID_ARG
     assert f(FAKE, 1, 1, 8, 8, None, 128, 2, FAKE, FAKE, FAKE, FAKE, None) == sas.SAS_ERR_UNSUPPORTED
-    assert f(FAKE, 1, 1, 2000, 2000, None, 64, 2, FAKE, FAKE, FAKE, FAKE, None) == sas.SAS_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 1, 16386, 16386, None, 64, 2, FAKE, FAKE, FAKE, FAKE, None) == sas.SAS_ERR_UNSUPPORTED
     assert f(FAKE, 1, 1, 8, 8, None, 64, 2, None, FAKE, None, FAKE, None) == sas.SAS_ERR_INVALID_ARG
 
 
 def test_bwd_and_decode_workspace_queries(L):
-    assert L.sas_attn_bwd_workspace_size(sas.SAS_BF16, 1, 100, 4, 2, 128, 2) == 0
+    assert L.sas_attn_bwd_workspace_size(sas.SAS_BF16, 1, 0, 4, 2, 128, 2) == 0
+    assert L.sas_attn_bwd_workspace_size(sas.SAS_BF16, 1, 100, 4, 2, 128, 2) > 0      # partial last block
     assert L.sas_attn_bwd_workspace_size(sas.SAS_BF16, 1, 128, 4, 2, 128, 2) > 0
+    # the tensor-core backward packs block and slot into 16 bits each: 32767 blocks at most
+    assert L.sas_attn_bwd_workspace_size(sas.SAS_BF16, 1, 32767 * 64, 4, 2, 128, 2) > 0
+    assert L.sas_attn_bwd_workspace_size(sas.SAS_BF16, 1, 32767 * 64 + 1, 4, 2, 128, 2) == 0
+    assert L.sas_attn_bwd_varlen_workspace_size(sas.SAS_BF16, 3, 100, 250, 4, 2, 128, 2) > 0
+    assert L.sas_attn_bwd_varlen_workspace_size(sas.SAS_BF16, 3, 100, 0, 4, 2, 128, 2) == 0
     assert L.sas_decode_workspace_size(4, 32, 8, 128, 32) > 0
     assert L.sas_decode_workspace_size(4, 32, 8, 64, 32) == 0
     # too-small workspace is rejected on the host
@@ -97,3 +103,23 @@ def test_decode_rejects_bad_arguments(L):
     assert f(*bad) == sas.SAS_ERR_UNSUPPORTED
     bad = list(args); bad[19] = ctypes.c_void_p(0x10010)  # workspace alignment
     assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+
+
+def test_varlen_rejects_bad_arguments(L):
+    f = L.sas_attn_fwd_varlen
+    args = [sas.SAS_BF16, FAKE, FAKE, FAKE, FAKE, 3, 100, 250, 4, 2, 128, 64, 2, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE,
+            None]
+    bad = list(args); bad[4] = None                       # no cu_seqlens
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[7] = 0                          # no token rows
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[6] = 0                          # max_seqlen 0
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[8] = 3                          # Hq % Hkv
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    sel = L.sas_select_varlen
+    assert sel(FAKE, 3, 2, 2, 2, None, 64, 2, FAKE, FAKE, FAKE, FAKE, None) == sas.SAS_ERR_INVALID_ARG
+    b = L.sas_attn_bwd_varlen
+    r = b(sas.SAS_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None,
+          3, 100, 250, 4, 2, 128, 64, 2, 0.1, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0x10000), 1 << 30, None)
+    assert r == sas.SAS_ERR_INVALID_ARG

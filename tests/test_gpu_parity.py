@@ -76,7 +76,7 @@ def test_select_full_workloads(name):
     _select_checks(s, cfg.K, gsel, O.prefill_history(NQB))
 
 
-@pytest.mark.parametrize("R", [200, 700])     # one-warp rows, and one-CTA rows (> 512 history)
+@pytest.mark.parametrize("R", [200, 700, 2000])   # one-warp rows; one-CTA rows (radix select) beyond 512
 def test_select_adversarial_ties(R):
     rng = np.random.default_rng(5)
     B, H = 2, 3
@@ -118,6 +118,12 @@ SMALL = [
     ("bf16-K0", "bf16", 1, 512, 4, 1, 128, 0, 1.0),
     ("bf16-dense", "bf16", 1, 512, 4, 1, 128, 8, 1.0),
     ("bf16-one-block", "bf16", 2, 64, 8, 2, 128, 4, 1.0),
+    # lengths that are not a multiple of 64 (a partial last block)
+    ("bf16-S100-g4", "bf16", 2, 100, 8, 2, 128, 3, 1.0),
+    ("f32-S229-d64", "f32", 1, 229, 2, 1, 64, 2, 1.0),
+    ("bf16-S1000-g5", "bf16", 1, 1000, 10, 2, 128, 4, 2.0),
+    ("bf16-S65-d64", "bf16", 1, 65, 4, 2, 64, 2, 1.0),
+    ("bf16-S1", "bf16", 2, 1, 8, 2, 128, 2, 1.0),
 ]
 
 
@@ -130,7 +136,7 @@ def _small_inputs(dtype, B, S, Hq, Hkv, D, K, std, seed):
 def test_fwd_bwd_small(case):
     name, dtype, B, S, Hq, Hkv, D, K, std = case
     cfg, x = _small_inputs(dtype, B, S, Hq, Hkv, D, K, std, seed=zlib.crc32(name.encode()) % 1000)
-    NQB = S // BLOCK
+    NQB = cfg.NQB
     sc = 1.0 / math.sqrt(D)
     xd = _dev(x)
     gsel = sas.select(_poisoned(x["s"]).cuda(), K)
@@ -232,10 +238,30 @@ def test_mixed_tile_items_sampled():
     _sampled_parity(cfg, [0, 1, 15, 64, 100, 127])
 
 
-def _sampled_parity(cfg, rows):
+def _dkv_picks(idx, cnt, b, h, G, NQB, rnd, budget, extra=()):
+    """Key blocks whose dk/dv the oracle recomputes: the last two, the block kept by the
+    most query blocks (the most kept one whose attending stripes fit the budget), blocks
+    given in ``extra``, and one attended by a handful of query blocks."""
+    picks = [NQB - 1, max(NQB - 2, 0)] + [j for j in extra if 0 <= j < NQB]
+    kept = np.bincount(idx[b, h][idx[b, h] >= 0].ravel(), minlength=NQB)
+    for j in np.argsort(-kept, kind="stable"):
+        if (kept[j] + 1) * G <= budget:
+            picks.append(int(j))
+            break
+    for j in rnd.sample(range(NQB), min(NQB, 40)):
+        if 3 <= len(_reverse(idx, cnt, b, h, j)) <= 12 and j not in picks:
+            picks.append(j)
+            break
+    return list(dict.fromkeys(picks))
+
+
+def _sampled_parity(cfg, rows, heads=2, dkv_extra=(), dkv_budget=800):
+    """Full-size run on the GPU; the oracle recomputes sampled stripes one by one: o, lse
+    and dq of the given query blocks (all heads of the sampled KV heads), their ds rows, and
+    dk/dv of at least four key blocks per sampled KV head."""
     x = inputs.make_prefill(cfg)
     xd = _dev(x)
-    NQB, G, D = cfg.NQB, cfg.G, cfg.D
+    NQB, G, D, S = cfg.NQB, cfg.G, cfg.D, cfg.S
     sc = 1.0 / math.sqrt(D)
     gsel = sas.select(xd["s"], cfg.K)
     o, lse = sas.attn_fwd(xd["q"], xd["k"], xd["v"], *gsel[:3], sc)
@@ -246,33 +272,30 @@ def _sampled_parity(cfg, rows):
     idx, cnt, lg, _ = _select_checks(x["s"], cfg.K, gsel, O.prefill_history(NQB))
     rnd = random.Random(cfg.seed + 1)
     b = cfg.B - 1
-    h = rnd.randrange(cfg.Hkv)
-    stripes = [(b, h * G + g, i) for i in rows for g in range(G)]
-    ro, rlse = O.attn_fwd(x["q"], x["k"], x["v"], idx, cnt, lg, sc, stripes=stripes)
-    rdq, _, _, rds, _ = O.attn_bwd(x["q"], x["k"], x["v"], x["do"], idx, cnt, lg, x["s"], sc, stripes=stripes)
-    for (bb, hq, i) in stripes:
-        rs = slice(i * 64, (i + 1) * 64)
-        check_out(o[bb, rs, hq], ro[bb, rs, hq], "bf16", f"o[{bb},{i},{hq}]")
-        check_out(lse[bb, hq, rs], rlse[bb, hq, rs], "bf16", f"lse[{bb},{i},{hq}]")
-    dq_s = np.stack([np64(dq[bb, i * 64:(i + 1) * 64, hq]) for bb, hq, i in stripes])
-    rdq_s = np.stack([rdq[bb, i * 64:(i + 1) * 64, hq] for bb, hq, i in stripes])
-    check_grad(dq_s, rdq_s, "bf16", "dq (sampled stripes)")
-    ds_s = np.stack([np64(ds[b, h, i, :NQB]) for i in rows])
-    rds_s = np.stack([rds[b, h, i, :NQB] for i in rows])
-    check_grad(ds_s, rds_s, "bf16", "ds (sampled rows)")
-    # dk/dv: key blocks whose attending stripes are few enough to recompute
-    picks = [NQB - 1, NQB - 2]
-    for j in rnd.sample(range(1, NQB - 2), 40):      # one key block several query blocks attend
-        if 3 <= len(_reverse(idx, cnt, b, h, j)) <= 12:
-            picks.append(j)
-            break
-    for j in picks:
-        att = _reverse(idx, cnt, b, h, j)
-        kst = [(b, h * G + g, i) for i in att for g in range(G)]
-        _, rdk, rdv, _, _ = O.attn_bwd(x["q"], x["k"], x["v"], x["do"], idx, cnt, lg, x["s"], sc, stripes=kst)
-        ks = slice(j * 64, (j + 1) * 64)
-        check_grad(dk[b, ks, h], rdk[b, ks, h], "bf16", f"dk block {j}")
-        check_grad(dv[b, ks, h], rdv[b, ks, h], "bf16", f"dv block {j}")
+    for h in rnd.sample(range(cfg.Hkv), min(heads, cfg.Hkv)):
+        stripes = [(b, h * G + g, i) for i in rows for g in range(G)]
+        ro, rlse = O.attn_fwd(x["q"], x["k"], x["v"], idx, cnt, lg, sc, stripes=stripes)
+        rdq, _, _, rds, _ = O.attn_bwd(x["q"], x["k"], x["v"], x["do"], idx, cnt, lg, x["s"], sc, stripes=stripes)
+        for (bb, hq, i) in stripes:
+            rs = O.block_rows(i, S)
+            check_out(o[bb, rs, hq], ro[bb, rs, hq], "bf16", f"{cfg.name} o[{bb},{i},{hq}]")
+            check_out(lse[bb, hq, rs], rlse[bb, hq, rs], "bf16", f"{cfg.name} lse[{bb},{i},{hq}]")
+        dq_s = np.concatenate([np64(dq[bb, O.block_rows(i, S), hq]) for bb, hq, i in stripes])
+        rdq_s = np.concatenate([rdq[bb, O.block_rows(i, S), hq] for bb, hq, i in stripes])
+        check_grad(dq_s, rdq_s, "bf16", f"{cfg.name} dq (sampled stripes, KV head {h})")
+        ds_s = np.stack([np64(ds[b, h, i, :NQB]) for i in rows])
+        rds_s = np.stack([rds[b, h, i, :NQB] for i in rows])
+        check_grad(ds_s, rds_s, "bf16", f"{cfg.name} ds (sampled rows, KV head {h})")
+        picks = _dkv_picks(idx, cnt, b, h, G, NQB, rnd, dkv_budget, dkv_extra)
+        assert len(picks) >= 4 or NQB < 4
+        for j in picks:
+            att = _reverse(idx, cnt, b, h, j)
+            kst = [(b, h * G + g, i) for i in att for g in range(G)]
+            _, rdk, rdv, _, _ = O.attn_bwd(x["q"], x["k"], x["v"], x["do"], idx, cnt, lg, x["s"], sc, stripes=kst)
+            ks = O.block_rows(j, S)
+            check_grad(dk[b, ks, h], rdk[b, ks, h], "bf16", f"{cfg.name} dk block {j} (KV head {h}, {len(att)} rows)")
+            check_grad(dv[b, ks, h], rdv[b, ks, h], "bf16", f"{cfg.name} dv block {j} (KV head {h}, {len(att)} rows)")
+    return idx, cnt
 
 
 # ---------------------------------------------------------------------------

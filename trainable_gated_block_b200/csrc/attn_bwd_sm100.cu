@@ -24,6 +24,12 @@
 // S and dP are computed twice (once per kernel) instead of once; in exchange
 // nothing is reduced through global memory and dq/dk/dv are deterministic.
 //
+// Sequence b occupies token rows start_b .. start_b + len_b - 1 (a dense batch
+// or a packed batch of different lengths); its last block may be partial.
+// Query rows past the end get P = dS = 0 (they are read by the Q/dO boxes
+// and dropped), key rows past the end get no dK/dV store, and items of blocks
+// past the end are skipped by every role.
+//
 // Barrier discipline: every mbarrier phase is waited on in order by its
 // consumer (a parity wait is exact only within one phase of the barrier), so
 // "buffer is free again" barriers are waited on before every reuse of the
@@ -56,6 +62,8 @@ constexpr uint32_t kHi = sm100::sdesc_hi(1024);   // high descriptor word: 8-row
 // ------------------------------------------------------------------ shared
 struct Params {
     int B, S, Hq, Hkv, G, K, NQB, n_items, ntile;
+    const int32_t* cu;      // packed sequence bounds [B + 1], or nullptr (dense)
+    long long T;            // token rows of q/k/v/dO
     const int32_t* idx;
     const int32_t* cnt;
     const float* log_gate;
@@ -143,8 +151,10 @@ struct Bars {
 };
 
 struct Item {
-    int b, h, i, t, c, nb;
+    int b, h, i, t, c, nb, len;
     long long row;     // selection row (b, h, i)
+    long long start;   // first token row of the sequence
+    bool skip;         // query block past the sequence's end
 };
 
 __device__ __forceinline__ Item item_of(const Params& p, int id) {
@@ -158,9 +168,20 @@ __device__ __forceinline__ Item item_of(const Params& p, int id) {
     it.h = bh % p.Hkv;
     it.b = bh / p.Hkv;
     it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
-    it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));
+    const SeqRange sr = seq_range(p.cu, it.b, p.S, p.T, nullptr);
+    it.start = sr.start;
+    it.len = sr.len;
+    it.skip = it.i * 64 >= it.len;
+    it.c = it.skip ? 0 : max(0, min(p.cnt[it.row], min(p.K, it.i)));
     it.nb = it.c + 1;
     return it;
+}
+
+// This CTA's next item at or after `id` (stride gridDim.x) that is not past
+// its sequence's end; every role walks the same list.
+__device__ __forceinline__ int live_item(const Params& p, int id) {
+    while (id < p.n_items && item_of(p, id).skip) id += gridDim.x;
+    return id;
 }
 
 struct Blk {
@@ -243,19 +264,22 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     const int hq = it.h * p.G + (slot < p.G ? slot : 0);
                     for (int a = 0; a < 2; ++a) {
                         const uint32_t off = a * kTileAtom + s * kBox;
-                        tma_load_3d(smem + kOffQs + off, &map_q, &bars->qs_full, a * 64, hq, it.b * p.S + it.i * 64);
+                        tma_load_3d(smem + kOffQs + off, &map_q, &bars->qs_full, a * 64, hq, (int)(it.start + it.i * 64));
                         tma_load_3d(smem + kOffQs + kTile + off, &map_do, &bars->qs_full, a * 64, hq,
-                                    it.b * p.S + it.i * 64);
+                                    (int)(it.start + it.i * 64));
                     }
                 }
                 ++qn;
                 q_pending = true;
                 return true;
             };
-            bool ok = blockIdx.x >= p.n_items || load_qd(blockIdx.x);
-            for (int id = blockIdx.x; id < p.n_items && ok && !*abort; id += gridDim.x) {
+            if (p.cu != nullptr)           // check the packed bounds once (flags a bad sequence)
+                for (int bb = 0; bb < p.B; ++bb) seq_range(p.cu, bb, p.S, p.T, p.status);
+            const int first = live_item(p, blockIdx.x);
+            bool ok = first >= p.n_items || load_qd(first);
+            for (int id = first; id < p.n_items && ok && !*abort; id = live_item(p, id + gridDim.x)) {
                 const Item it = item_of(p, id);
-                const int nxt = id + gridDim.x;
+                const int nxt = live_item(p, id + gridDim.x);
                 const int k_next = min(1, it.nb - 1);   // the next item's Q/dO goes out after this block
                 for (int k = 0; k < it.nb && ok; ++k, ++kb) {
                     const int st = kb % kNS;
@@ -265,11 +289,11 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
                     mbar_expect_tx(&bars->k_full[st], 2 * kBox);
                     for (int a = 0; a < 2; ++a)
                         tma_load_3d(smem + kOffKV + st * kStage + a * kBlkAtom, &map_k, &bars->k_full[st], a * 64, it.h,
-                                    it.b * p.S + bk.j * 64);
+                                    (int)(it.start + bk.j * 64));
                     mbar_expect_tx(&bars->v_full[st], 2 * kBox);
                     for (int a = 0; a < 2; ++a)
                         tma_load_3d(smem + kOffKV + st * kStage + kBlk + a * kBlkAtom, &map_v, &bars->v_full[st],
-                                    a * 64, it.h, it.b * p.S + bk.j * 64);
+                                    a * 64, it.h, (int)(it.start + bk.j * 64));
                     last_kv[st] = (int)kb;
                     if (k == k_next && nxt < p.n_items) ok = load_qd(nxt);
                 }
@@ -298,7 +322,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             const uint32_t d_tm = tmem + kTmS + 128 * u + (is_s ? 0u : 64u);
             const uint32_t b_off = is_s ? 0u : kBlk;
             uint32_t n_mine = 0;
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
+            for (int id = live_item(p, blockIdx.x); id < p.n_items && ok; id = live_item(p, id + gridDim.x), ++qn) {
                 const Item it = item_of(p, id);
                 // this item's Q and dO are in TMEM
                 if (!(ok = mbar_wait_warp(&bars->qt_full, qn & 1, abort, p.status))) break;
@@ -329,7 +353,7 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             // dQ += dS K (SS: A = dS tile of the block's warpgroup, B = K MN-major)
             const uint32_t id_dq = idesc_bf16(128, kD, false, true);
             uint32_t ds_n[2] = {0, 0};
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
+            for (int id = live_item(p, blockIdx.x); id < p.n_items && ok; id = live_item(p, id + gridDim.x), ++qn) {
                 const Item it = item_of(p, id);
                 for (int k = 0; k < it.nb && ok; ++k, ++kb) {
                     const int u = kb & 1, st = kb % kNS;
@@ -391,15 +415,16 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             mbar_arrive(&bars->qt_full);
             return true;
         };
-        if (blockIdx.x < p.n_items) ok = copy_qd(0);
-        for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x, ++qn) {
+        if (live_item(p, blockIdx.x) < p.n_items) ok = copy_qd(0);
+        for (int id = live_item(p, blockIdx.x); id < p.n_items && ok; id = live_item(p, id + gridDim.x), ++qn) {
             const Item it = item_of(p, id);
             const int slot = 2 * it.t + slot_in_tile;
-            const bool row_ok = slot < p.G;
-            const int hq = it.h * p.G + (row_ok ? slot : 0);
+            // rows of an absent head, or past the sequence's end, contribute nothing
+            const bool row_ok = slot < p.G && it.i * 64 + r_in < it.len;
+            const int hq = it.h * p.G + (slot < p.G ? slot : 0);
             const long long lrow = ((long long)it.b * p.Hq + hq) * p.S + (long long)it.i * 64 + r_in;
-            const float lse2 = p.lse[lrow] * kLog2e;
-            const float drs = p.Dr[lrow] * p.sm_scale;
+            const float lse2 = row_ok ? p.lse[lrow] * kLog2e : 0.f;
+            const float drs = row_ok ? p.Dr[lrow] * p.sm_scale : 0.f;
             // this warpgroup's blocks: stream positions kb + k with (kb + k) % 2 == u
             int k = (int)((u - (int)(kb & 1)) & 1);
             Blk nxt;
@@ -442,11 +467,11 @@ dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUt
             kb += it.nb;
             // the next item's Q / dO go into TMEM first, so that its S / dP start
             // while this item's dQ is written out
-            if (id + (int)gridDim.x < p.n_items && !(ok = copy_qd(qn + 1))) break;
+            if (live_item(p, id + gridDim.x) < p.n_items && !(ok = copy_qd(qn + 1))) break;
             // dQ of the item: warpgroup u writes dims [64 u, 64 u + 64) of its rows
             if (!(ok = mbar_wait(&bars->dq_full, qn & 1, abort, p.status))) break;
             tc_fence_after();
-            const long long orow = ((long long)it.b * p.S + (long long)it.i * 64 + r_in) * p.Hq + hq;
+            const long long orow = (it.start + (long long)it.i * 64 + r_in) * p.Hq + hq;
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 uint32_t ov[32];
@@ -510,17 +535,29 @@ struct Bars {
     int abort;
 };
 
-__device__ __forceinline__ void item_of(const Params& p, int id, int& b, int& h, int& j, long long& bh) {
-    j = id % p.NQB;
+// Item (b, h, j) and its sequence's token range; len = 0 marks an item whose
+// key block lies past the sequence's end (skipped by every role).
+struct KItem {
+    int b, h, j, len;
+    long long bh, start;
+};
+__device__ __forceinline__ KItem item_of(const Params& p, int id) {
+    KItem it;
+    it.j = id % p.NQB;
     const int r = id / p.NQB;
-    h = r % p.Hkv;
-    b = r / p.Hkv;
-    bh = (long long)b * p.Hkv + h;
+    it.h = r % p.Hkv;
+    it.b = r / p.Hkv;
+    it.bh = (long long)it.b * p.Hkv + it.h;
+    const SeqRange sr = seq_range(p.cu, it.b, p.S, p.T, nullptr);
+    it.start = sr.start;
+    it.len = it.j * 64 < sr.len ? sr.len : 0;
+    return it;
 }
 
-__device__ __forceinline__ int n_entries(const Params& p, long long bh, int j) {
-    const int n = p.rcount[bh * p.NQB + j];
-    return max(1, min(n, p.NQB - j));
+__device__ __forceinline__ int n_entries(const Params& p, const KItem& it) {
+    if (it.len == 0) return 0;
+    const int n = p.rcount[it.bh * p.NQB + it.j];
+    return max(1, min(n, p.NQB - it.j));
 }
 
 // Item of this CTA's round r, or -1 past the end: the items sorted by
@@ -544,24 +581,25 @@ struct StepMeta {
     int slot, idxv;
     float lg, lse, drow;
 };
-__device__ __forceinline__ StepMeta step_meta(const Params& p, int ent, int b, int h, long long bh, int j, int m,
-                                              int row) {
+__device__ __forceinline__ StepMeta step_meta(const Params& p, int ent, const KItem& it, int m, int row) {
     StepMeta s;
     const int t = m % p.ntile;
+    const int j = it.j;
     int i = ent >> 16;
     s.slot = ent & 0xFFFF;
     s.in_range = i >= j && i < p.NQB;
     if (!s.in_range) i = j;
     s.cur = (i == j);
-    const long long sidx = (bh * p.NQB + i) * p.K + min(s.slot, p.K - 1);
+    const long long sidx = (it.bh * p.NQB + i) * p.K + min(s.slot, p.K - 1);
     s.idxv = s.cur ? j : __ldg(p.idx + sidx);
     s.lg = s.cur ? 0.f : __ldg(p.log_gate + sidx);
     const int hs = 2 * t + (row >> 6);
-    s.row_ok = hs < p.G;
-    const int hq = h * p.G + (s.row_ok ? hs : 0);
-    const long long lrow = ((long long)b * p.Hq + hq) * p.S + (long long)i * 64 + (row & 63);
-    s.lse = __ldg(p.lse + lrow);
-    s.drow = __ldg(p.Dr + lrow);
+    // rows of an absent head, or past the sequence's end, contribute nothing
+    s.row_ok = hs < p.G && i * 64 + (row & 63) < it.len;
+    const int hq = it.h * p.G + (hs < p.G ? hs : 0);
+    const long long lrow = ((long long)it.b * p.Hq + hq) * p.S + (long long)i * 64 + (row & 63);
+    s.lse = s.row_ok ? __ldg(p.lse + lrow) : 0.f;
+    s.drow = s.row_ok ? __ldg(p.Dr + lrow) : 0.f;
     return s;
 }
 
@@ -608,19 +646,20 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         if (lane == 0) {
             uint32_t item_it = 0, g = 0, npos = 0;      // npos: Q / dO tiles issued
             bool kv_issued = false;
-            for (int r = 0, id; (id = item_at(p, r)) >= 0 && !*abort; ++r, ++item_it) {
-                int b, h, j;
-                long long bh;
-                item_of(p, id, b, h, j, bh);
-                const int n = n_entries(p, bh, j);
+            for (int r = 0, id; (id = item_at(p, r)) >= 0 && !*abort; ++r) {
+                const KItem it = item_of(p, id);
+                const int n = n_entries(p, it);
+                if (n == 0) continue;                   // key block past the sequence's end
+                const int h = it.h, j = it.j;
                 if (!mbar_wait(&bars->kv_empty, (item_it & 1) ^ 1, abort, p.status)) break;
+                ++item_it;
                 mbar_expect_tx(&bars->kv_full, 4 * kBox);
                 for (int a = 0; a < 2; ++a) {
-                    tma_load_3d(smem + kOffK + a * kBlkAtom, &map_k, &bars->kv_full, a * 64, h, b * p.S + j * 64);
-                    tma_load_3d(smem + kOffV + a * kBlkAtom, &map_v, &bars->kv_full, a * 64, h, b * p.S + j * 64);
+                    tma_load_3d(smem + kOffK + a * kBlkAtom, &map_k, &bars->kv_full, a * 64, h, (int)(it.start + j * 64));
+                    tma_load_3d(smem + kOffV + a * kBlkAtom, &map_v, &bars->kv_full, a * 64, h, (int)(it.start + j * 64));
                 }
                 kv_issued = true;
-                const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
+                const int32_t* list = p.rlist + (it.bh * p.NQB + j) * p.NQB;
                 bool ok = true;
                 for (int e = 0; e < n && ok; ++e) {
                     int i = __ldg(list + e) >> 16;
@@ -642,7 +681,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                                 const int hq = h * p.G + (hs < p.G ? hs : 0);
                                 for (int a = 0; a < 2; ++a)
                                     tma_load_3d(smem + kOffRing + sl * kTile + a * kTileAtom + s * kBox, mp, fb, a * 64,
-                                                hq, b * p.S + i * 64);
+                                                hq, (int)(it.start + i * 64));
                             }
                             ++npos;
                         }
@@ -669,12 +708,11 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             const bool is_s = slot == 0;
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t kv_lo = sdesc_lo(s_base + (is_s ? kOffK : kOffV), 16);
-            for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r, ++item_it) {
-                int b, h, j;
-                long long bh;
-                item_of(p, id, b, h, j, bh);
-                const int N = n_entries(p, bh, j) * p.ntile;
+            for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r) {
+                const int N = n_entries(p, item_of(p, id)) * p.ntile;
+                if (N == 0) continue;                   // key block past the sequence's end
                 if (!(ok = mbar_wait_warp(&bars->kv_full, item_it & 1, abort, p.status))) break;
+                ++item_it;
                 for (int m = 0; m < N && ok; ++m, ++g) {
                     const uint32_t pos = 2 * g + (is_s ? 0 : 1);
                     const int sl = pos % kSlots;
@@ -706,13 +744,12 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             const uint32_t id_t = idesc_bf16(128, 64, true, true);
             const uint32_t acc = tmem + (is_v ? kTmAccV : kTmAccK);
             const uint32_t pb_lo = sdesc_lo(s_base + (is_v ? kOffP : kOffDS), kRowTile);
-            for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r, ++item_it) {
-                int b, h, j;
-                long long bh;
-                item_of(p, id, b, h, j, bh);
-                const int N = n_entries(p, bh, j) * p.ntile;
+            for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r) {
+                const int N = n_entries(p, item_of(p, id)) * p.ntile;
+                if (N == 0) continue;                   // key block past the sequence's end
                 // the drain of the previous item has read the accumulators
                 if (!(ok = mbar_wait_warp(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
+                ++item_it;
                 for (int m = 0; m < N && ok; ++m, ++g) {
                     if (!(ok = mbar_wait_warp(&bars->pds_full, g & 1, abort, p.status))) break;
                     tc_fence_after();
@@ -743,18 +780,18 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         uint8_t* bufS = smem + kOffDS;
         uint32_t item_it = 0, g = 0;
         bool ok = true;
-        for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r, ++item_it) {
-            int b, h, j;
-            long long bh;
-            item_of(p, id, b, h, j, bh);
-            const int N = n_entries(p, bh, j) * p.ntile;
-            const int32_t* list = p.rlist + (bh * p.NQB + j) * p.NQB;
+        for (int r = 0, id; (id = item_at(p, r)) >= 0 && ok; ++r) {
+            const KItem it = item_of(p, id);
+            const int N = n_entries(p, it) * p.ntile;
+            if (N == 0) continue;                       // key block past the sequence's end
+            const int j = it.j;
+            const int32_t* list = p.rlist + (it.bh * p.NQB + j) * p.NQB;
             // metadata pipeline: entry of step m + 2 and loads of step m + 1 in flight
             int ent2 = (1 < N) ? __ldg(list + 1 / p.ntile) : 0;
-            StepMeta nxt = step_meta(p, __ldg(list), b, h, bh, j, 0, row);
+            StepMeta nxt = step_meta(p, __ldg(list), it, 0, row);
             for (int m = 0; m < N; ++m, ++g) {
                 const StepMeta sm = nxt;
-                if (m + 1 < N) nxt = step_meta(p, ent2, b, h, bh, j, m + 1, row);
+                if (m + 1 < N) nxt = step_meta(p, ent2, it, m + 1, row);
                 if (m + 2 < N) ent2 = __ldg(list + (m + 2) / p.ntile);
                 const int buf = g & 1;
                 if (!(ok = mbar_wait(&bars->s_full[buf], (g >> 1) & 1, abort, p.status))) break;
@@ -780,13 +817,16 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 mbar_arrive(&bars->pds_full);
             }
             if (!ok) break;
-            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim index)
+            // drain: warpgroup 0 writes dV, warpgroup 1 writes dK (TMEM lane = head-dim index);
+            // keys past the sequence's end are not stored
             if (!(ok = mbar_wait(&bars->acc_full, item_it & 1, abort, p.status))) break;
+            ++item_it;
             tc_fence_after();
             {
                 const int d = row;
-                __nv_bfloat16* out = (w == 0 ? p.dv : p.dk) + ((long long)b * p.S + (long long)j * 64) * p.Hkv * kD +
-                                     (long long)h * kD + d;
+                const int keys = min(64, it.len - j * 64);
+                __nv_bfloat16* out = (w == 0 ? p.dv : p.dk) + (it.start + (long long)j * 64) * p.Hkv * kD +
+                                     (long long)it.h * kD + d;
                 const long long key_stride = (long long)p.Hkv * kD;
 #pragma unroll 1
                 for (int qt = 0; qt < 4; ++qt) {
@@ -794,8 +834,14 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                     tmem_ld16(tmem + lane_base + (w == 0 ? kTmAccV : kTmAccK) + 16 * qt, v0);
                     tmem_wait_ld();
                     __nv_bfloat16* o2 = out + 16 * qt * key_stride;
+                    if (16 * qt + 16 <= keys) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) o2[u * key_stride] = __float2bfloat16_rn(__uint_as_float(v0[u]));
+                        for (int u = 0; u < 16; ++u) o2[u * key_stride] = __float2bfloat16_rn(__uint_as_float(v0[u]));
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u)
+                            if (16 * qt + u < keys) o2[u * key_stride] = __float2bfloat16_rn(__uint_as_float(v0[u]));
+                    }
                 }
             }
             tc_fence_before();
@@ -813,13 +859,15 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 }  // namespace dkv
 
 // ================================================================ helpers
-// Dr = rowsum(O * dO) over D = 128 for every (b, t, hq) row; Dr as [B, Hq, S].
-// HBM-bound: a warp takes 8 consecutive rows, 16 lanes per row with 16-byte
-// loads, all eight loads of a lane issued before any is used.
+// Dr = rowsum(O * dO) over D = 128 for every (token, hq) row; Dr as [B, Hq, S]
+// (rows of no sequence are skipped). HBM-bound: a warp takes 8 consecutive
+// rows, 16 lanes per row with 16-byte loads, all eight loads of a lane issued
+// before any is used.
 constexpr int kDotRowsPerWarp = 8;
 __global__ void __launch_bounds__(256) dot_rows_kernel(const __nv_bfloat16* __restrict__ o,
-                                                       const __nv_bfloat16* __restrict__ dout, long long rows, int S,
-                                                       int Hq, float* __restrict__ Dr) {
+                                                       const __nv_bfloat16* __restrict__ dout, long long rows, int B,
+                                                       int S, int Hq, const int32_t* __restrict__ cu,
+                                                       float* __restrict__ Dr) {
     const long long w0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kDotRowsPerWarp;
     const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
     uint4 a[kDotRowsPerWarp / 2], c[kDotRowsPerWarp / 2];
@@ -845,11 +893,10 @@ __global__ void __launch_bounds__(256) dot_rows_kernel(const __nv_bfloat16* __re
 #pragma unroll
         for (int m = 8; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
         const long long row = w0 + 2 * r + half;
-        if (l16 == 0 && row < rows) {
+        int b, t;
+        if (l16 == 0 && row < rows && token_seq(cu, B, S, row / Hq, b, t)) {
             const int hq = (int)(row % Hq);
-            const long long bt = row / Hq;
-            const long long b = bt / S, t = bt % S;
-            Dr[(b * Hq + hq) * S + t] = acc;
+            Dr[((long long)b * Hq + hq) * S + t] = acc;
         }
     }
 }
@@ -897,13 +944,15 @@ __global__ void __launch_bounds__(1024) dkv_order_kernel(const int32_t* __restri
 }
 
 __global__ void rev_fill_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int rows, int NQB,
-                                int K, int16_t* __restrict__ slotmap) {
+                                int K, int Hkv, const int32_t* __restrict__ cu, int S, long long T,
+                                int16_t* __restrict__ slotmap) {
     const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     const int i = (int)(row % NQB);
     const long long bh = row / NQB;
-    const int c = max(0, min(cnt[row], min(K, i)));
+    const int len = seq_range(cu, (int)(bh / Hkv), S, T, nullptr).len;
+    const int c = i * 64 < len ? max(0, min(cnt[row], min(K, i))) : 0;
     for (int k = lane; k < c; k += 32) {
         const int j = idx[row * K + k];
         if (j >= 0 && j < i) slotmap[(bh * NQB + j) * NQB + i] = (int16_t)(k + 1);
@@ -942,7 +991,7 @@ struct Ws {
 };
 
 Ws carve(void* w, int B, int S, int Hq, int Hkv, int K) {
-    const int NQB = S / 64;
+    const int NQB = (S + 63) / 64;
     char* p = static_cast<char*>(w);
     Ws r;
     r.Dr = reinterpret_cast<float*>(p);
@@ -962,7 +1011,7 @@ Ws carve(void* w, int B, int S, int Hq, int Hkv, int K) {
 }  // namespace
 
 size_t bwd_sm100_workspace(int B, int S, int Hq, int Hkv, int K) {
-    const int NQB = S / 64;
+    const int NQB = (S + 63) / 64;
     return align256(sizeof(float) * (size_t)B * Hq * S) +
            align256(sizeof(float) * (size_t)B * Hkv * NQB * (size_t)(K > 0 ? K : 1)) +
            align256(sizeof(int16_t) * (size_t)B * Hkv * NQB * NQB) +
@@ -971,8 +1020,8 @@ size_t bwd_sm100_workspace(int B, int S, int Hq, int Hkv, int K) {
 
 cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     const AttnArgs& a = bw.a;
-    const int NQB = a.S / 64, G = a.Hq / a.Hkv;
-    const long long rows = (long long)a.B * a.S;
+    const int NQB = (a.S + 63) / 64, G = a.Hq / a.Hkv;
+    const long long rows = a.T;
     CUtensorMap mq, mdo, mk, mv;
     if (!make_head_map(&mq, a.q, rows, a.Hq, kD) || !make_head_map(&mdo, bw.dout, rows, a.Hq, kD) ||
         !make_head_map(&mk, a.k, rows, a.Hkv, kD) || !make_head_map(&mv, a.v, rows, a.Hkv, kD))
@@ -984,9 +1033,9 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     if ((e = cudaMemsetAsync(ws.slotmap, 0, sizeof(int16_t) * (size_t)bhq * NQB, st)) != cudaSuccess) return e;
     const long long drows = rows * a.Hq;
     const long long dwarps = (drows + kDotRowsPerWarp - 1) / kDotRowsPerWarp;
-    dot_rows_kernel<<<(unsigned)((dwarps + 7) / 8), 256, 0, st>>>((const __nv_bfloat16*)bw.o,
-                                                                  (const __nv_bfloat16*)bw.dout, drows, a.S, a.Hq, ws.Dr);
-    rev_fill_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(a.idx, a.cnt, bhq, NQB, a.K, ws.slotmap);
+    dot_rows_kernel<<<(unsigned)((dwarps + 7) / 8), 256, 0, st>>>(
+        (const __nv_bfloat16*)bw.o, (const __nv_bfloat16*)bw.dout, drows, a.B, a.S, a.Hq, a.cu, ws.Dr);
+    rev_fill_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(a.idx, a.cnt, bhq, NQB, a.K, a.Hkv, a.cu, a.S, a.T, ws.slotmap);
     rev_list_kernel<<<(bhq + 7) / 8, 256, 0, st>>>(ws.slotmap, bhq, NQB, ws.rlist, ws.rcount);
     // buckets per head: 64, fewer when there are more than 128 (batch, KV head) pairs
     const int n_bh = a.B * a.Hkv;
@@ -1004,6 +1053,8 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     p.G = G;
     p.K = a.K;
     p.NQB = NQB;
+    p.cu = a.cu;
+    p.T = a.T;
     p.ntile = (G + 1) / 2;
     p.idx = a.idx;
     p.cnt = a.cnt;
@@ -1039,7 +1090,8 @@ cudaError_t launch_bwd_sm100(const BwdArgs& bw, cudaStream_t st) {
     dkv::dkv_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, dkv::kSmem, st>>>(mq, mdo, mk, mv, p);
     count_launches(2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return launch_ds_finalize(bw.s, bw.ld_s, bw.lse_s, a.idx, a.cnt, ws.gsum, a.B, a.Hkv, NQB, a.K, bw.ds, st);
+    return launch_ds_finalize(bw.s, bw.ld_s, bw.lse_s, a.idx, a.cnt, ws.gsum, a.B, a.Hkv, NQB, a.K, a.cu, a.S, a.T,
+                              bw.ds, st);
 }
 
 }  // namespace sas

@@ -9,6 +9,11 @@
 // 128-row Q tiles, each tile = 2 query heads x the 64 rows of block i. All
 // query heads of a GQA group share the kept blocks, so one K/V block feeds
 // both Q tiles. Persistent grid; items head by head, longest first within a head.
+// Sequence b occupies token rows start_b .. start_b + len_b - 1 (a dense batch,
+// or a packed batch of different lengths). Its last block may be partial: the
+// Q box reads past the sequence (those rows are computed and dropped), and the
+// keys past its end lie above every valid row, so the causal mask removes
+// them. Items of query blocks past a sequence's end are skipped by every role.
 //
 // One step = one kept block (64 keys). Warp roles (352 threads):
 //   warp 0      TMA producer: the Q tiles once per item, then K and V of one
@@ -96,6 +101,8 @@ __device__ __forceinline__ bool wait_count(const uint32_t* c, uint32_t target, v
 
 struct Params {
     int B, S, Hq, Hkv, G, K, NQB, ntg, n_items;
+    const int32_t* cu;                  // packed sequence bounds [B + 1], or nullptr (dense)
+    long long T;                        // token rows of q/k/v
     const int32_t* idx;
     const int32_t* cnt;
     const float* log_gate;
@@ -106,8 +113,9 @@ struct Params {
 };
 
 struct Item {
-    int b, h, i, tg, nt, c, nb;
-    long long row;
+    int b, h, i, tg, nt, c, nb, len;
+    long long row, start;               // selection row; first token row of the sequence
+    bool skip;                          // query block past the sequence's end
 };
 
 __device__ __forceinline__ Item item_of(const Params& p, int id) {
@@ -122,9 +130,20 @@ __device__ __forceinline__ Item item_of(const Params& p, int id) {
     it.b = bh / p.Hkv;
     it.nt = (4 * it.tg + 2 < p.G) ? 2 : 1;
     it.row = ((long long)it.b * p.Hkv + it.h) * p.NQB + it.i;
-    it.c = max(0, min(p.cnt[it.row], min(p.K, it.i)));
+    const SeqRange sr = seq_range(p.cu, it.b, p.S, p.T, nullptr);
+    it.start = sr.start;
+    it.len = sr.len;
+    it.skip = it.i * 64 >= it.len;
+    it.c = it.skip ? 0 : max(0, min(p.cnt[it.row], min(p.K, it.i)));
     it.nb = it.c + 1;
     return it;
+}
+
+// This CTA's next item at or after `id` (stride gridDim.x) that is not past
+// its sequence's end; every role walks the same list.
+__device__ __forceinline__ int live_item(const Params& p, int id) {
+    while (id < p.n_items && item_of(p, id).skip) id += gridDim.x;
+    return id;
 }
 
 // Block k of the item's list: kept blocks ascending, then the current block.
@@ -200,7 +219,9 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             uint32_t kv_it = 0, q_it = 0;
             int last_it[kNS] = {-1, -1, -1, -1};
             bool q_issued = false;
-            for (int id = blockIdx.x; id < p.n_items && !*abort; id += gridDim.x) {
+            if (p.cu != nullptr)           // check the packed bounds once (flags a bad sequence)
+                for (int b = 0; b < p.B; ++b) seq_range(p.cu, b, p.S, p.T, p.status);
+            for (int id = live_item(p, blockIdx.x); id < p.n_items && !*abort; id = live_item(p, id + gridDim.x)) {
                 const Item it = item_of(p, id);
                 if (p.cnt[it.row] != it.c) flag_status(p.status, kStatusBadData);
                 if (!mbar_wait(&bars->q_empty, (q_it & 1) ^ 1, abort, p.status)) break;
@@ -211,7 +232,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         const int hq = it.h * p.G + (slot < p.G ? slot : 0);
                         for (int a = 0; a < 2; ++a)
                             tma_load_3d(smem + kOffQ + t * kQTile + a * kQAtom + s * kBox, &map_q, &bars->q_full,
-                                        a * 64, hq, it.b * p.S + it.i * 64);
+                                        a * 64, hq, (int)(it.start + it.i * 64));
                     }
                 q_issued = true;
                 ++q_it;
@@ -223,11 +244,11 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     mbar_expect_tx(&bars->k_full[st], 2 * kBox);
                     for (int a = 0; a < 2; ++a)
                         tma_load_3d(smem + kOffKV + st * kStage + a * kBlkAtom, &map_k, &bars->k_full[st], a * 64,
-                                    it.h, it.b * p.S + m.j * 64);
+                                    it.h, (int)(it.start + m.j * 64));
                     mbar_expect_tx(&bars->v_full[st], 2 * kBox);
                     for (int a = 0; a < 2; ++a)
                         tma_load_3d(smem + kOffKV + st * kStage + kBlk + a * kBlkAtom, &map_v, &bars->v_full[st],
-                                    a * 64, it.h, it.b * p.S + m.j * 64);
+                                    a * 64, it.h, (int)(it.start + m.j * 64));
                     last_it[st] = (int)kv_it;
                 }
             }
@@ -263,7 +284,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 mma_commit(&bars->s_full[t][buf]);
             };
             bool ok = true;
-            for (int id = blockIdx.x; id < p.n_items && ok; id += gridDim.x) {
+            for (int id = live_item(p, blockIdx.x); id < p.n_items && ok; id = live_item(p, id + gridDim.x)) {
                 const Item it = item_of(p, id);
                 if (!(ok = mbar_wait(&bars->q_full, q_it & 1, abort, p.status))) break;
                 ++q_it;
@@ -341,7 +362,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const uint32_t tO = tT + 128;
         // pv_count[t]: PVs of this tile completed so far (published by the issuer)
         uint32_t s_it[2] = {0, 0}, pv_it = 0;
-        for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
+        for (int id = live_item(p, blockIdx.x); id < p.n_items; id = live_item(p, id + gridDim.x)) {
             const Item it = item_of(p, id);
             if (t >= it.nt) continue;
             const int slot = 4 * it.tg + 2 * t + slot_in_tile;
@@ -418,9 +439,9 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             pv_it += it.nb;
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const bool store = slot < p.G;
+            const bool store = slot < p.G && it.i * 64 + r_in < it.len;
             const int hq = it.h * p.G + slot;
-            const long long orow = ((long long)it.b * p.S + (long long)it.i * 64 + r_in) * p.Hq + hq;
+            const long long orow = (it.start + (long long)it.i * 64 + r_in) * p.Hq + hq;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 uint32_t ov[32];
@@ -458,7 +479,7 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
 cudaError_t launch_fwd_sm100(const AttnArgs& a, void* o, float* lse, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
-    const long long rows = (long long)a.B * a.S;
+    const long long rows = a.T;
     if (!make_head_map(&mq, a.q, rows, a.Hq, kD) || !make_head_map(&mk, a.k, rows, a.Hkv, kD) ||
         !make_head_map(&mv, a.v, rows, a.Hkv, kD))
         return cudaErrorInvalidValue;
@@ -469,7 +490,9 @@ cudaError_t launch_fwd_sm100(const AttnArgs& a, void* o, float* lse, cudaStream_
     p.Hkv = a.Hkv;
     p.G = a.Hq / a.Hkv;
     p.K = a.K;
-    p.NQB = a.S / 64;
+    p.NQB = (a.S + 63) / 64;
+    p.cu = a.cu;
+    p.T = a.T;
     p.ntg = ((p.G + 1) / 2 + 1) / 2;
     p.n_items = a.B * a.Hkv * p.NQB * p.ntg;
     p.idx = a.idx;

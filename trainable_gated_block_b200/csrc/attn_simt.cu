@@ -11,7 +11,10 @@
 // This is the fp32 dtype path (tensor cores would round the operands). One
 // CTA of 128 threads owns a 64-row stripe (b, hq, query block i): thread
 // pairs split the head dimension of one query row. Key/value tiles of 64
-// rows are staged in shared memory.
+// rows are staged in shared memory. Sequence b occupies token rows start_b ..
+// start_b + len_b - 1; a partial last block is staged with zero rows past the
+// end, its rows past the end are neither stored nor given gradient, and CTAs
+// of blocks past the end return at once.
 #include "common.cuh"
 #include "launch.h"
 
@@ -21,12 +24,13 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kChunk = 16;              // keys per online-softmax update
 
-// Loads a 64 x D tile (rows `row0..row0+63` of head h) into shared memory as fp32.
+// Loads a 64 x D tile (rows `row0..row0+63` of head h; rows from `nrows` on
+// read as zero) into shared memory as fp32.
 template <typename T, int D>
-__device__ __forceinline__ void load_tile(float* dst, const T* src, long long row0, int H, int h) {
+__device__ __forceinline__ void load_tile(float* dst, const T* src, long long row0, int H, int h, int nrows) {
     for (int e = threadIdx.x; e < kBlock * D; e += kThreads) {
         const int r = e / D, d = e % D;
-        dst[r * (D + 1) + d] = Elem<T>::load(src + ((row0 + r) * H + h) * (long long)D + d);
+        dst[r * (D + 1) + d] = r < nrows ? Elem<T>::load(src + ((row0 + r) * H + h) * (long long)D + d) : 0.f;
     }
 }
 
@@ -38,7 +42,7 @@ __device__ __forceinline__ int tile_at(const int32_t* sel, int n_sel, int t, int
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                int S, int Hq, int Hkv, int K,
+                int S, int Hq, int Hkv, int K, const int32_t* __restrict__ cu, long long Trows,
                 const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
                 const float* __restrict__ log_gate, float sm_scale,
                 T* __restrict__ o, float* __restrict__ lse, int* status) {
@@ -47,14 +51,17 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     float* Ks = smem;                               // [64][D+1]
     float* Vs = Ks + kBlock * (D + 1);              // [64][D+1]
     const int i = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
-    const int NQB = S / kBlock, G = Hq / Hkv, h = hq / G;
+    const int NQB = (S + kBlock - 1) / kBlock, G = Hq / Hkv, h = hq / G;
     const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
-    const long long t = (long long)b * S + (long long)i * kBlock + row;     // token row
+    const SeqRange sr = seq_range(cu, b, S, Trows, threadIdx.x == 0 ? status : nullptr);
+    if (i * kBlock >= sr.len) return;               // block past the sequence's end
+    const bool row_ok = i * kBlock + row < sr.len;
+    const long long t = sr.start + (long long)i * kBlock + row;     // token row
 
     float qr[HD], acc[HD];
 #pragma unroll
     for (int d = 0; d < HD; ++d) {
-        qr[d] = Elem<T>::load(q + (t * Hq + hq) * D + half * HD + d) * sm_scale * kLog2e;
+        qr[d] = row_ok ? Elem<T>::load(q + (t * Hq + hq) * D + half * HD + d) * sm_scale * kLog2e : 0.f;
         acc[d] = 0.f;
     }
     const long long sel_row = ((long long)(b * Hkv + h) * NQB + i);
@@ -71,8 +78,9 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         if (!ok) flag_status(status, kStatusBadData);
         __syncthreads();
         if (ok) {
-            load_tile<T, D>(Ks, k, (long long)b * S + (long long)j * kBlock, Hkv, h);
-            load_tile<T, D>(Vs, v, (long long)b * S + (long long)j * kBlock, Hkv, h);
+            const int nr = min(kBlock, sr.len - j * kBlock);
+            load_tile<T, D>(Ks, k, sr.start + (long long)j * kBlock, Hkv, h, nr);
+            load_tile<T, D>(Vs, v, sr.start + (long long)j * kBlock, Hkv, h, nr);
         }
         __syncthreads();
         if (!ok) continue;
@@ -107,6 +115,7 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             }
         }
     }
+    if (!row_ok) return;
     const float inv = 1.f / l;
 #pragma unroll
     for (int d = 0; d < HD; ++d) Elem<T>::store(o + (t * Hq + hq) * D + half * HD + d, acc[d] * inv);
@@ -126,27 +135,27 @@ struct BwdWs {
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline BwdWs carve(void* ws, int B, int S, int Hq, int Hkv, int D, int K) {
+inline BwdWs carve(void* ws, int B, int S, long long T, int Hq, int Hkv, int D, int K) {
     char* p = static_cast<char*>(ws);
     BwdWs w;
-    const int NQB = S / kBlock;
+    const int NQB = (S + kBlock - 1) / kBlock;
     w.Dr = reinterpret_cast<float*>(p); p += align256(sizeof(float) * (size_t)B * Hq * S);
     w.gsum = reinterpret_cast<float*>(p); p += align256(sizeof(float) * (size_t)B * Hkv * NQB * (size_t)(K > 0 ? K : 1));
-    w.dk = reinterpret_cast<float*>(p); p += align256(sizeof(float) * (size_t)B * S * Hkv * D);
+    w.dk = reinterpret_cast<float*>(p); p += align256(sizeof(float) * (size_t)T * Hkv * D);
     w.dv = reinterpret_cast<float*>(p);
     return w;
 }
 
 template <typename T, int D>
-__global__ void bwd_dot_kernel(const T* __restrict__ o, const T* __restrict__ dout, int B, int S, int Hq,
-                               float* __restrict__ Dr) {
-    // One warp per (b, token, hq) row; Dr stored as [B, Hq, S].
+__global__ void bwd_dot_kernel(const T* __restrict__ o, const T* __restrict__ dout, int B, int S, long long Trows,
+                               int Hq, const int32_t* __restrict__ cu, float* __restrict__ Dr) {
+    // One warp per (token, hq) row; Dr stored as [B, Hq, S] (rows of no sequence skipped).
     const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (w >= (long long)B * S * Hq) return;
+    if (w >= Trows * Hq) return;
     const int hq = (int)(w % Hq);
-    const long long bt = w / Hq;
-    const int b = (int)(bt / S), t = (int)(bt % S);
+    int b, t;
+    if (!token_seq(cu, B, S, w / Hq, b, t)) return;
     float acc = 0.f;
     for (int d = lane; d < D; d += 32) acc = fmaf(Elem<T>::load(o + w * D + d), Elem<T>::load(dout + w * D + d), acc);
     acc = warp_sum(acc);
@@ -157,7 +166,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const T* __restrict__ dout, const float* __restrict__ lse,
-                int S, int Hq, int Hkv, int K,
+                int S, int Hq, int Hkv, int K, const int32_t* __restrict__ cu, long long Trows,
                 const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
                 const float* __restrict__ log_gate, float sm_scale,
                 T* __restrict__ dq, BwdWs ws, int* status) {
@@ -172,12 +181,16 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     float* red = dSs + kBlock * (kBlock + 1);       // [4] warp partial sums
 
     const int i = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
-    const int NQB = S / kBlock, G = Hq / Hkv, h = hq / G;
+    const int NQB = (S + kBlock - 1) / kBlock, G = Hq / Hkv, h = hq / G;
     const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
-    const long long t = (long long)b * S + (long long)i * kBlock + row;
+    const SeqRange sr = seq_range(cu, b, S, Trows, nullptr);
+    if (i * kBlock >= sr.len) return;               // block past the sequence's end
+    const int nrows = min(kBlock, sr.len - i * kBlock);
+    const bool row_ok = row < nrows;
+    const long long t = sr.start + (long long)i * kBlock + row;
 
-    load_tile<T, D>(Qs, q, (long long)b * S + (long long)i * kBlock, Hq, hq);
-    load_tile<T, D>(dOs, dout, (long long)b * S + (long long)i * kBlock, Hq, hq);
+    load_tile<T, D>(Qs, q, sr.start + (long long)i * kBlock, Hq, hq, nrows);
+    load_tile<T, D>(dOs, dout, sr.start + (long long)i * kBlock, Hq, hq, nrows);
     __syncthreads();
     float qr[HD], dor[HD], dqa[HD];
 #pragma unroll
@@ -186,8 +199,8 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         dor[d] = dOs[row * (D + 1) + half * HD + d];
         dqa[d] = 0.f;
     }
-    const float lse2 = lse[((long long)b * Hq + hq) * S + (long long)i * kBlock + row] * kLog2e;
-    const float Drow = ws.Dr[((long long)b * Hq + hq) * S + (long long)i * kBlock + row];
+    const float lse2 = row_ok ? lse[((long long)b * Hq + hq) * S + (long long)i * kBlock + row] * kLog2e : 0.f;
+    const float Drow = row_ok ? ws.Dr[((long long)b * Hq + hq) * S + (long long)i * kBlock + row] : 0.f;
 
     const long long sel_row = ((long long)(b * Hkv + h) * NQB + i);
     int n_sel = cnt[sel_row];
@@ -201,9 +214,10 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         const bool ok = cur || (j >= 0 && j < i);
         if (!ok) flag_status(status, kStatusBadData);
         __syncthreads();
+        const int nk = min(kBlock, sr.len - j * kBlock);     // keys of block j inside the sequence
         if (ok) {
-            load_tile<T, D>(Ks, k, (long long)b * S + (long long)j * kBlock, Hkv, h);
-            load_tile<T, D>(Vs, v, (long long)b * S + (long long)j * kBlock, Hkv, h);
+            load_tile<T, D>(Ks, k, sr.start + (long long)j * kBlock, Hkv, h, nk);
+            load_tile<T, D>(Vs, v, sr.start + (long long)j * kBlock, Hkv, h, nk);
         }
         __syncthreads();
         if (!ok) continue;
@@ -217,7 +231,7 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
             for (int d = 0; d < HD; ++d) { sdot = fmaf(qr[d], kr[d], sdot); pdot = fmaf(dor[d], vr[d], pdot); }
             sdot += __shfl_xor_sync(0xffffffffu, sdot, 1);
             pdot += __shfl_xor_sync(0xffffffffu, pdot, 1);
-            const bool masked = cur && u > row;
+            const bool masked = (cur && u > row) || !row_ok;
             const float p = masked ? 0.f : exp2f(sdot + bias - lse2);
             const float dsv = p * (pdot - Drow);
 #pragma unroll
@@ -239,7 +253,7 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         {
             constexpr int DC = 16;                      // head-dim columns per pass
             const int u = threadIdx.x >> 1;
-            const long long krow = ((long long)b * S + (long long)j * kBlock + u) * Hkv + h;
+            const long long krow = (sr.start + (long long)j * kBlock + u) * Hkv + h;
 #pragma unroll 1
             for (int d0 = 0; d0 < HD; d0 += DC) {
                 float dka[DC], dva[DC];
@@ -253,10 +267,12 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
 #pragma unroll
                     for (int d = 0; d < DC; ++d) { dka[d] = fmaf(dsv, qrow[d], dka[d]); dva[d] = fmaf(pv, drow[d], dva[d]); }
                 }
+                if (u < nk) {                       // keys past the sequence's end: no store
 #pragma unroll
-                for (int d = 0; d < DC; ++d) {
-                    atomicAdd(ws.dk + krow * D + half * HD + d0 + d, dka[d] * sm_scale);
-                    atomicAdd(ws.dv + krow * D + half * HD + d0 + d, dva[d]);
+                    for (int d = 0; d < DC; ++d) {
+                        atomicAdd(ws.dk + krow * D + half * HD + d0 + d, dka[d] * sm_scale);
+                        atomicAdd(ws.dv + krow * D + half * HD + d0 + d, dva[d]);
+                    }
                 }
             }
         }
@@ -264,6 +280,7 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         if (!cur && threadIdx.x == 0)
             atomicAdd(ws.gsum + sel_row * K + tt, red[0] + red[1] + red[2] + red[3]);
     }
+    if (!row_ok) return;
 #pragma unroll
     for (int d = 0; d < HD; ++d) Elem<T>::store(dq + (t * Hq + hq) * D + half * HD + d, dqa[d] * sm_scale);
 }
@@ -279,12 +296,16 @@ __global__ void cast_kernel(const float* __restrict__ src, T* __restrict__ dst, 
 // ds from the per-block gate gradients (shared by every backward path).
 __global__ void ds_finalize_kernel(const float* __restrict__ s, int ld_s, const float* __restrict__ lse_s,
                                    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
-                                   const float* __restrict__ gsum, int rows, int NQB, int K,
-                                   float* __restrict__ ds) {
+                                   const float* __restrict__ gsum, int rows, int NQB, int K, int Hkv,
+                                   const int32_t* __restrict__ cu, int S, long long T, float* __restrict__ ds) {
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (row >= rows) return;
     const int i = (int)(row % NQB);
+    if (i * kBlock >= seq_range(cu, (int)(row / NQB / Hkv), S, T, nullptr).len) {
+        for (int j = lane; j < ld_s; j += 32) ds[row * (long long)ld_s + j] = 0.f;   // padding row
+        return;
+    }
     const int c = min(max(cnt[row], 0), min(K, i));
     float tot = 0.f;
     for (int m = lane; m < c; m += 32) tot += gsum[row * K + m];
@@ -303,9 +324,10 @@ __global__ void ds_finalize_kernel(const float* __restrict__ s, int ld_s, const 
 
 cudaError_t launch_ds_finalize(const float* s, int ld_s, const float* lse_s, const int32_t* idx,
                                const int32_t* cnt, const float* gsum, int B, int Hkv, int NQB, int K,
-                               float* ds, cudaStream_t st) {
+                               const int32_t* cu, int S, long long T, float* ds, cudaStream_t st) {
     const int rows = B * Hkv * NQB;
-    ds_finalize_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, ld_s, lse_s, idx, cnt, gsum, rows, NQB, K, ds);
+    ds_finalize_kernel<<<(rows + 7) / 8, 256, 0, st>>>(s, ld_s, lse_s, idx, cnt, gsum, rows, NQB, K, Hkv, cu, S, T,
+                                                       ds);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -316,8 +338,8 @@ static cudaError_t fwd_go(const AttnArgs& a, void* o, float* lse, cudaStream_t s
     auto kern = fwd_simt_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.S / kBlock, a.Hq, a.B);
-    kern<<<grid, kThreads, sm, st>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.S, a.Hq, a.Hkv, a.K,
+    dim3 grid((a.S + kBlock - 1) / kBlock, a.Hq, a.B);
+    kern<<<grid, kThreads, sm, st>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.S, a.Hq, a.Hkv, a.K, a.cu, a.T,
                                      a.idx, a.cnt, a.log_gate, a.sm_scale, (T*)o, lse, a.status);
     count_launches(1);
     return cudaGetLastError();
@@ -328,27 +350,28 @@ cudaError_t launch_fwd_simt(const AttnArgs& a, bool bf16, void* o, float* lse, c
     return a.D == 64 ? fwd_go<float, 64>(a, o, lse, st) : fwd_go<float, 128>(a, o, lse, st);
 }
 
-size_t bwd_simt_workspace(int B, int S, int Hq, int Hkv, int D, int K) {
-    const int NQB = S / kBlock;
+size_t bwd_simt_workspace(int B, int S, long long T, int Hq, int Hkv, int D, int K) {
+    const int NQB = (S + kBlock - 1) / kBlock;
     return align256(sizeof(float) * (size_t)B * Hq * S) +
            align256(sizeof(float) * (size_t)B * Hkv * NQB * (size_t)(K > 0 ? K : 1)) +
-           2 * align256(sizeof(float) * (size_t)B * S * Hkv * D);
+           2 * align256(sizeof(float) * (size_t)T * Hkv * D);
 }
 
 template <typename T, int D>
 static cudaError_t bwd_go(const BwdArgs& p, cudaStream_t st) {
     const AttnArgs& a = p.a;
-    BwdWs ws = carve(p.workspace, a.B, a.S, a.Hq, a.Hkv, a.D, a.K);
-    const int NQB = a.S / kBlock;
+    BwdWs ws = carve(p.workspace, a.B, a.S, a.T, a.Hq, a.Hkv, a.D, a.K);
+    const int NQB = (a.S + kBlock - 1) / kBlock;
     cudaError_t e;
     e = cudaMemsetAsync(ws.gsum, 0, sizeof(float) * (size_t)a.B * a.Hkv * NQB * (size_t)(a.K > 0 ? a.K : 1), st);
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(ws.dk, 0, sizeof(float) * (size_t)a.B * a.S * a.Hkv * D, st);
+    e = cudaMemsetAsync(ws.dk, 0, sizeof(float) * (size_t)a.T * a.Hkv * D, st);
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(ws.dv, 0, sizeof(float) * (size_t)a.B * a.S * a.Hkv * D, st);
+    e = cudaMemsetAsync(ws.dv, 0, sizeof(float) * (size_t)a.T * a.Hkv * D, st);
     if (e != cudaSuccess) return e;
-    const long long rows = (long long)a.B * a.S * a.Hq;
-    bwd_dot_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)p.o, (const T*)p.dout, a.B, a.S, a.Hq, ws.Dr);
+    const long long rows = a.T * a.Hq;
+    bwd_dot_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)p.o, (const T*)p.dout, a.B, a.S, a.T,
+                                                                     a.Hq, a.cu, ws.Dr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t sm = sizeof(float) * (4 * kBlock * (D + 1) + 2 * kBlock * (kBlock + 1) + 4);
     auto kern = bwd_simt_kernel<T, D>;
@@ -356,15 +379,16 @@ static cudaError_t bwd_go(const BwdArgs& p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     dim3 grid(NQB, a.Hq, a.B);
     kern<<<grid, kThreads, sm, st>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)p.dout, p.lse,
-                                     a.S, a.Hq, a.Hkv, a.K, a.idx, a.cnt, a.log_gate, a.sm_scale,
+                                     a.S, a.Hq, a.Hkv, a.K, a.cu, a.T, a.idx, a.cnt, a.log_gate, a.sm_scale,
                                      (T*)p.dq, ws, a.status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const long long n = (long long)a.B * a.S * a.Hkv * D;
+    const long long n = a.T * a.Hkv * D;
     cast_kernel<T><<<1184, 256, 0, st>>>(ws.dk, (T*)p.dk, n);
     cast_kernel<T><<<1184, 256, 0, st>>>(ws.dv, (T*)p.dv, n);
     count_launches(4);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return launch_ds_finalize(p.s, p.ld_s, p.lse_s, a.idx, a.cnt, ws.gsum, a.B, a.Hkv, NQB, a.K, p.ds, st);
+    return launch_ds_finalize(p.s, p.ld_s, p.lse_s, a.idx, a.cnt, ws.gsum, a.B, a.Hkv, NQB, a.K, a.cu, a.S, a.T, p.ds,
+                              st);
 }
 
 cudaError_t launch_bwd_simt(const BwdArgs& p, bool bf16, cudaStream_t st) {

@@ -17,6 +17,52 @@ __device__ __forceinline__ void flag_status(int* status, int code) {
     if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Token rows of sequence b of a batch. Dense batches (cu == nullptr) hold B
+// sequences of S tokens, sequence b at rows b*S .. b*S+S-1; packed batches
+// hold sequence b at rows cu[b] .. cu[b+1]-1, with S the longest length.
+// Packed bounds that are out of range (negative, longer than S, or past the
+// T rows) are flagged and the sequence is treated as empty.
+struct SeqRange {
+    long long start;
+    int len;
+};
+__device__ __forceinline__ SeqRange seq_range(const int32_t* cu, int b, int S, long long T, int* status) {
+    SeqRange r;
+    if (cu == nullptr) {
+        r.start = (long long)b * S;
+        r.len = S;
+        return r;
+    }
+    const int a = __ldg(cu + b), e = __ldg(cu + b + 1);
+    r.start = a;
+    r.len = e - a;
+    if (a < 0 || r.len < 0 || r.len > S || (long long)e > T) {
+        flag_status(status, kStatusBadData);
+        r.start = 0;
+        r.len = 0;
+    }
+    return r;
+}
+
+// Sequence and position of token row `tok` (binary search over cu for packed
+// batches). Returns false for a row that belongs to no sequence.
+__device__ __forceinline__ bool token_seq(const int32_t* cu, int B, int S, long long tok, int& b, int& t) {
+    if (cu == nullptr) {
+        b = (int)(tok / S);
+        t = (int)(tok % S);
+        return b < B;
+    }
+    int lo = 0, hi = B;                      // find the last b with cu[b] <= tok
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)__ldg(cu + mid) <= tok) lo = mid; else hi = mid;
+    }
+    b = lo;
+    const long long st = __ldg(cu + lo), en = __ldg(cu + lo + 1);
+    t = (int)(tok - st);
+    return tok >= st && tok < en && t < S;
+}
+
 template <typename T> struct Elem;
 template <> struct Elem<float> {
     static __device__ __forceinline__ float load(const float* p) { return *p; }

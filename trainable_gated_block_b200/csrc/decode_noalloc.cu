@@ -16,14 +16,16 @@
 //     call wrote. Nothing in it has to start at zero: each split writes its
 //     whole partial before the combine step reads it. Calls that overlap on
 //     the GPU (different streams, or threads without ordering) race on it.
-//   * the first call on a device looks up the array's device address (once
-//     per device, with that device current); make that first call before any
-//     stream capture.
+//   * the first call on a device looks up the array's device address (with
+//     that device current) and caches it with the id of the current context;
+//     it is looked up again only when another context is current (after a
+//     cudaDeviceReset). Make the first call on a device, and the first call
+//     after a reset, before any stream capture.
 // No cudaMalloc, cudaFree or allocating library routine is called here.
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdio>
+#include <mutex>
 
 #include "../../include/sas.h"
 #include "launch.h"
@@ -37,7 +39,11 @@ constexpr size_t kScratchBytes = size_t(16) << 20;     // 16 MiB
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
+void* g_scratch_addr[kMaxDevices] = {};
+
+cudaError_t scratch_lookup(void** out) { return cudaGetSymbolAddress(out, g_decode_scratch); }
 
 }  // namespace
 
@@ -62,17 +68,18 @@ extern "C" sas_status sas_decode_paged_noalloc(const void* q, const void* k_cach
         sas::set_last_error("sas_decode_paged_noalloc: no usable current CUDA device");
         return SAS_ERR_CUDA;
     }
-    void* ptr = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (ptr == nullptr) {
-        e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-        if (e != cudaSuccess || ptr == nullptr) {
-            char msg[256];
-            snprintf(msg, sizeof msg, "sas_decode_paged_noalloc: cudaGetSymbolAddress failed: %s",
-                     cudaGetErrorString(e));
-            sas::set_last_error(msg);
-            return SAS_ERR_CUDA;
-        }
-        g_scratch_addr[dev].store(ptr, std::memory_order_release);
+    // Set-up: the array's device address, looked up with this device current
+    // and cached together with the id of the context it belongs to (after a
+    // cudaDeviceReset the device gets a new context and the array a new
+    // address, so the lookup is repeated whenever the context changes).
+    void* ptr = nullptr;
+    e = sas::cached_symbol_address(dev, &g_scratch_mu, g_scratch_ctx, g_scratch_addr, scratch_lookup, &ptr);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "sas_decode_paged_noalloc: cudaGetSymbolAddress failed: %s",
+                 cudaGetErrorString(e));
+        sas::set_last_error(msg);
+        return SAS_ERR_CUDA;
     }
     // Same validation and kernels as the workspace entry point, on the static scratch.
     return sas_decode_paged(q, k_cache, v_cache, num_pages, page_table, max_pages, kv_len, N, Hq, Hkv, D,

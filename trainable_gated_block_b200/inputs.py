@@ -55,7 +55,7 @@ class PrefillConfig:
 
     @property
     def NQB(self) -> int:
-        return self.S // BLOCK
+        return (self.S + BLOCK - 1) // BLOCK
 
     @property
     def torch_dtype(self):
@@ -105,8 +105,10 @@ def _randn(shape, g, dtype, chunk_elems=1 << 26):
 
 
 def make_prefill(cfg: PrefillConfig, seed: int | None = None, with_do: bool = True):
-    """Return a dict of CPU tensors: q, k, v ([B,S,H,D]), s ([B,Hkv,NQB,NQB] fp32), do."""
-    assert cfg.S % BLOCK == 0 and cfg.Hq % cfg.Hkv == 0
+    """Return a dict of CPU tensors: q, k, v ([B,S,H,D]), s ([B,Hkv,NQB,NQB] fp32), do.
+
+    S need not be a multiple of 64 (NQB = ceil(S/64)) except for stand-in scores."""
+    assert cfg.Hq % cfg.Hkv == 0 and (cfg.scores != "standin" or cfg.S % BLOCK == 0)
     g = torch.Generator().manual_seed(cfg.seed if seed is None else seed)
     dt = cfg.torch_dtype
     B, S, Hq, Hkv, D, NQB = cfg.B, cfg.S, cfg.Hq, cfg.Hkv, cfg.D, cfg.NQB
@@ -123,9 +125,35 @@ def make_prefill(cfg: PrefillConfig, seed: int | None = None, with_do: bool = Tr
     else:
         raise ValueError(cfg.scores)
     out = dict(q=q, k=k, v=v, s=s.contiguous())
+    if cfg.scores == "standin":
+        out["noise"] = noise            # the random part of the stand-in scores
     if with_do:
         out["do"] = _randn((B, S, Hq, D), g, dt)
     return out
+
+
+def make_varlen(lengths, Hq: int, Hkv: int, D: int, dtype: str = "bf16", score_std: float = 1.0,
+                seed: int = 0):
+    """A packed batch of sequences of the given lengths (CPU tensors).
+
+    Returns q, do [T,Hq,D], k, v [T,Hkv,D] (T = sum of lengths), cu_seqlens int32
+    [B+1], max_seqlen, and scores s [B,Hkv,R,R] fp32 ~ N(0, score_std), R = the
+    blocks of the longest sequence. Draw order: q, k, v, scores, dO.
+    """
+    g = torch.Generator().manual_seed(seed)
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    T = int(sum(lengths))
+    B = len(lengths)
+    max_seqlen = max(lengths)
+    R = (max_seqlen + BLOCK - 1) // BLOCK
+    cu = torch.zeros(B + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    q = _randn((T, Hq, D), g, dt)
+    k = _randn((T, Hkv, D), g, dt)
+    v = _randn((T, Hkv, D), g, dt)
+    s = (_randn((B, Hkv, R, R), g, torch.float32).double() * score_std).float()
+    do = _randn((T, Hq, D), g, dt)
+    return dict(q=q, k=k, v=v, s=s.contiguous(), do=do, cu_seqlens=cu, max_seqlen=max_seqlen)
 
 
 def make_decode(cfg: DecodeConfig, seed: int | None = None):
@@ -162,3 +190,20 @@ def make_decode(cfg: DecodeConfig, seed: int | None = None):
     s = _randn((N, Hkv, cfg.max_hist), g, torch.float32)
     return dict(q=q, k_cache=k_cache, v_cache=v_cache, page_table=page_table,
                 kv_len=kv_len, s=s)
+
+
+def make_decode_device(N: int, ctx: int, Hq: int, Hkv: int, D: int, seed: int, device):
+    """Decode inputs drawn on the device, for timing studies whose caches are too large to
+    draw on the host (batch 8 at 512K holds 17 GB of pages). Every sequence holds ``ctx``
+    cached tokens plus one new token (kv_len = ctx + 1); its ctx/64 + 1 pages are scattered
+    by one seeded permutation of all pages. Scores s [N, Hkv, ctx/64] ~ N(0,1)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    pages = ctx // BLOCK + 1
+    total = N * pages
+    page_table = torch.randperm(total, generator=g, device=device).to(torch.int32).view(N, pages).contiguous()
+    kv_len = torch.full((N,), ctx + 1, dtype=torch.int32, device=device)
+    q = torch.randn((N, Hq, D), generator=g, device=device).to(torch.bfloat16)
+    k_cache = torch.randn((total, Hkv, BLOCK, D), generator=g, device=device, dtype=torch.bfloat16)
+    v_cache = torch.randn((total, Hkv, BLOCK, D), generator=g, device=device, dtype=torch.bfloat16)
+    s = torch.randn((N, Hkv, ctx // BLOCK), generator=g, device=device)
+    return dict(q=q, k_cache=k_cache, v_cache=v_cache, page_table=page_table, kv_len=kv_len, s=s)

@@ -145,7 +145,13 @@ TRAFFIC_SOURCES = {
     "sas_attn_bwd": ["attn_bwd_sm100.cu", "attn_simt.cu", "sm100.cuh", "common.cuh"],
 }
 DRAM_TRAFFIC = {
-    # workload -> entry point -> (bytes per call, sha256[:16] of the sources above)
+    # workload -> entry point -> (bytes per call, sha256[:16] of the sources above);
+    # the backward's figure sums Dr, dq and dk/dv (its index and ds kernels, about
+    # 40 MB, are not in the capture)
+    "qwen3-8b-32k": {
+        "sas_attn_fwd": (641096192, "cf7b2d7377903d8d"),
+        "sas_attn_bwd": (5673958656, "5045d376589e51c9"),
+    },
 }
 
 

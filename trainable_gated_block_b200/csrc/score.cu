@@ -16,7 +16,8 @@
 //    (fp32, in the workspace). Reads q and k once: HBM-bound.
 //  * score_select_kernel - one warp per selection row (b, h, i), eight rows of
 //    one (b, h) per CTA. Chunks of 32 pooled keys are staged in shared memory
-//    (one row per lane, padded against bank conflicts) and every lane forms
+//    (one row per lane, 16-byte rows padded against bank conflicts, read as
+//    float4) and every lane forms
 //    the dot product of its key with the warp's pooled query, so that lane l
 //    holds s[i][32 e + l] - the register layout of the warp-row selection,
 //    which runs next (select_row.cuh). s is written once (the backward's
@@ -89,15 +90,18 @@ pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
 // (b, h) = blockIdx.y; lane l of the warp computes j = 32 e + l for every
 // chunk e below `chunks`. The pooled keys of chunk e are staged by the CTA.
 template <int E, bool kSelect>
-__global__ void __launch_bounds__(kRowsPerCta * 32)
+__global__ void __launch_bounds__(kRowsPerCta * 32, 3)     // three CTAs per SM: 85 registers at most
 score_select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int NQB, int D, float inv_sqrt_d,
                     const float* __restrict__ noise, int ld_noise, float* __restrict__ s, int ld_s, int K,
                     int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ log_gate,
                     float* __restrict__ lse_s, int* status) {
     extern __shared__ float sm[];
-    float* kc = sm;                                            // [32][D + 1] pooled keys of a chunk
+    // two [32][D + 4] buffers of pooled keys (chunk e in buffer e & 1): rows 16-byte aligned,
+    // and the +4 padding keeps the eight lanes of each quarter-warp 128-bit load on distinct
+    // banks. Chunk e + 1 is loaded into registers while chunk e is used.
+    const int ldk = D + 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* qrow = sm + 32 * (D + 1) + warp * D;                // this warp's pooled query
+    float* qrow = sm + 2 * 32 * ldk + warp * D;                // this warp's pooled query
     const long long bh = blockIdx.y;
     const int i = blockIdx.x * kRowsPerCta + warp;
     const bool live = i < NQB;
@@ -106,28 +110,50 @@ score_select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, 
     if (live)
         for (int d = lane; d < D; d += 32) qrow[d] = qp[row * D + d];
     const int chunks = kSelect ? E : (i_max + 31) / 32;
+    const int used = (i_max + 31) / 32;                        // chunks holding some j < i_max
+    constexpr int kPer = 32 * 128 / 4 / (kRowsPerCta * 32);    // float4 of a chunk per thread (D = 128)
+    float4 nxt[kPer];
+    auto fetch = [&](int e) {                                  // chunk e -> registers
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int t = threadIdx.x + u * kRowsPerCta * 32;
+            const int r = t / (D / 4), d4 = t % (D / 4);
+            nxt[u] = (t < 8 * D && e * 32 + r < i_max)
+                         ? reinterpret_cast<const float4*>(kp + (bh * NQB + e * 32 + r) * D)[d4]
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto stash = [&](int e) {                                  // registers -> buffer e & 1
+        float* kc = sm + (e & 1) * 32 * ldk;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int t = threadIdx.x + u * kRowsPerCta * 32;
+            if (t < 8 * D) reinterpret_cast<float4*>(kc + (t / (D / 4)) * ldk)[t % (D / 4)] = nxt[u];
+        }
+    };
     float val[kSelect ? E : 1];
 #pragma unroll
     for (int e = 0; e < (kSelect ? E : 1); ++e) val[e] = -INFINITY;
+    if (used > 0) {
+        fetch(0);
+        stash(0);
+    }
     for (int e = 0; e < chunks; ++e) {
-        const int j0 = e * 32;
-        if (j0 < i_max) {                                      // the same for the whole CTA
-            __syncthreads();                                   // the previous chunk is consumed
-            for (int t = threadIdx.x; t < 32 * D; t += kRowsPerCta * 32) {
-                const int r = t / D, d = t % D;
-                kc[r * (D + 1) + d] = (j0 + r < i_max) ? kp[(bh * NQB + j0 + r) * D + d] : 0.f;
-            }
-            __syncthreads();
+        if (e < used) {                                        // the same for the whole CTA
+            if (e + 1 < used) fetch(e + 1);                    // in flight while chunk e is used
+            __syncthreads();                                   // chunk e is in its buffer
         }
-        const int j = j0 + lane;
+        const int j = e * 32 + lane;
         if (live && j < i) {
-            const float* kr = kc + lane * (D + 1);
+            const float4* kr = reinterpret_cast<const float4*>(sm + (e & 1) * 32 * ldk + lane * ldk);
+            const float4* qr = reinterpret_cast<const float4*>(qrow);
             float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;       // four chains
-            for (int d = 0; d < D; d += 4) {
-                a0 = fmaf(qrow[d], kr[d], a0);
-                a1 = fmaf(qrow[d + 1], kr[d + 1], a1);
-                a2 = fmaf(qrow[d + 2], kr[d + 2], a2);
-                a3 = fmaf(qrow[d + 3], kr[d + 3], a3);
+            for (int d4 = 0; d4 < D / 4; ++d4) {
+                const float4 kv = kr[d4], qv = qr[d4];
+                a0 = fmaf(qv.x, kv.x, a0);
+                a1 = fmaf(qv.y, kv.y, a1);
+                a2 = fmaf(qv.z, kv.z, a2);
+                a3 = fmaf(qv.w, kv.w, a3);
             }
             float v = ((a0 + a1) + (a2 + a3)) * inv_sqrt_d;
             if (noise != nullptr) v += __ldg(noise + row * (long long)ld_noise + j);
@@ -138,6 +164,7 @@ score_select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, 
                     if (ee == e) val[ee] = v;
             }
         }
+        if (e + 1 < used) stash(e + 1);                        // the other buffer: no one reads it now
     }
     if (kSelect && live) select_warp_row<kSelect ? E : 1>(val, i, K, row, idx, cnt, log_gate, lse_s, status);
 }
@@ -147,7 +174,7 @@ cudaError_t go_fused(const float* qp, const float* kp, int B, int Hkv, int NQB, 
                      int ld_noise, float* s, int ld_s, int K, int32_t* idx, int32_t* cnt, float* lg, float* lse_s,
                      int* status, cudaStream_t st) {
     const dim3 grid((NQB + kRowsPerCta - 1) / kRowsPerCta, B * Hkv);
-    const size_t sm = sizeof(float) * (32 * (D + 1) + kRowsPerCta * D);
+    const size_t sm = sizeof(float) * (2 * 32 * (D + 4) + kRowsPerCta * D);
     score_select_kernel<E, true><<<grid, kRowsPerCta * 32, sm, st>>>(qp, kp, NQB, D, inv, noise, ld_noise, s, ld_s,
                                                                      K, idx, cnt, lg, lse_s, status);
     count_launches(1);
@@ -306,7 +333,7 @@ cudaError_t launch_score_select(const ScoreArgs& a, cudaStream_t st) {
 #undef SAS_FUSED_ARGS
     // longer rows: scores first, then the CTA-per-row selection
     const dim3 grid((NQB + kRowsPerCta - 1) / kRowsPerCta, a.B * a.Hkv);
-    const size_t sm = sizeof(float) * (32 * (a.D + 1) + kRowsPerCta * a.D);
+    const size_t sm = sizeof(float) * (2 * 32 * (a.D + 4) + kRowsPerCta * a.D);
     score_select_kernel<1, false><<<grid, kRowsPerCta * 32, sm, st>>>(
         qp, kp, NQB, a.D, inv, a.noise, a.ld_noise, a.s, a.ld_s, a.K, a.idx, a.cnt, a.log_gate, a.lse_s, a.status);
     count_launches(1);

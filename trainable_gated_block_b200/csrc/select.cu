@@ -85,8 +85,9 @@ select_kernel(const float* __restrict__ s, int B, int Hkv, int n_rows, int ld_s,
 // j / (32 W), so the loads are coalesced). LSE by block reductions. The K-th
 // largest key T is found by a radix select: four passes over 8-bit digits,
 // most significant first; each pass histograms the digit of the keys that
-// still match the prefix found so far (shared-memory atomics), and one warp
-// scans the 256 bins from the top to find the digit holding the K-th key.
+// still match the prefix found so far (shared-memory atomics, one per group of
+// lanes of a warp holding the same digit), and one warp scans the 256 bins
+// from the top to find the digit holding the K-th key.
 // A kept key's output position is (# keys > T before it) + min(need,
 // # keys == T before it), so indices come out ascending.
 template <int E, int W>
@@ -99,7 +100,7 @@ select_cta_kernel(const float* __restrict__ s, int B, int Hkv, int n_rows, int l
     __shared__ float red_f[W];
     __shared__ unsigned hist[256];
     __shared__ unsigned sel_digit, sel_need;
-    __shared__ unsigned red_eq[2][W], red_gt[2][W];
+    __shared__ unsigned cnt_eq[E][W], cnt_gt[E][W], tot_eq[E], tot_gt[E];
     __shared__ int any_bad;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long row = blockIdx.x;
@@ -167,9 +168,14 @@ select_cta_kernel(const float* __restrict__ s, int B, int Hkv, int n_rows, int l
             for (int c = threadIdx.x; c < 256; c += NT) hist[c] = 0u;
             __syncthreads();
 #pragma unroll
-            for (int e = 0; e < E; ++e)
-                if (e * NT + (int)threadIdx.x < nh && (key[e] & mask) == prefix)
-                    atomicAdd(&hist[(key[e] >> shift) & 255u], 1u);
+            for (int e = 0; e < E; ++e) {
+                // scores crowd into a few digits (most keys share their top byte), so the
+                // lanes of a warp that hold the same digit add their count in one atomic
+                const bool in = e * NT + (int)threadIdx.x < nh && (key[e] & mask) == prefix;
+                const unsigned digit = in ? (key[e] >> shift) & 255u : 256u;
+                const unsigned peers = __match_any_sync(0xffffffffu, digit);
+                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+            }
             __syncthreads();
             if (warp == 0) {
                 // lane l owns bins 255 - 8l down to 248 - 8l (scanned from the top)
@@ -210,37 +216,57 @@ select_cta_kernel(const float* __restrict__ s, int B, int Hkv, int n_rows, int l
 
     const unsigned lt_mask = (1u << lane) - 1u;
     if (kk > 0) {
-        int eq_seen = 0, gt_seen = 0;
+        // Output position of a kept key = (# keys > T before it) + min(need, # keys == T before
+        // it), in index order j = e * NT + thread. Every warp publishes its per-chunk counts,
+        // warp e scans chunk e's counts over the warps, and the chunk totals are summed in order.
+        static_assert(E <= W, "one scanning warp per chunk");
 #pragma unroll
         for (int e = 0; e < E; ++e) {
             const bool valid = (e * NT + (int)threadIdx.x) < nh;
-            const bool eq = valid && key[e] == T;
-            const bool gtk = valid && key[e] > T;
-            const unsigned eq_ball = __ballot_sync(0xffffffffu, eq);
-            const unsigned gt_ball = __ballot_sync(0xffffffffu, gtk);
+            const unsigned eb = __ballot_sync(0xffffffffu, valid && key[e] == T);
+            const unsigned gb = __ballot_sync(0xffffffffu, valid && key[e] > T);
             if (lane == 0) {
-                red_eq[e & 1][warp] = __popc(eq_ball);
-                red_gt[e & 1][warp] = __popc(gt_ball);
+                cnt_eq[e][warp] = __popc(eb);
+                cnt_gt[e][warp] = __popc(gb);
             }
-            __syncthreads();
-            int eq_before = eq_seen, gt_before = gt_seen;
+        }
+        __syncthreads();
+        if (warp < E) {                       // warp e: exclusive prefix of chunk e over the warps
+            const unsigned ce = lane < W ? cnt_eq[warp][lane] : 0u, cg = lane < W ? cnt_gt[warp][lane] : 0u;
+            unsigned ie = ce, ig = cg;
 #pragma unroll
-            for (int w = 0; w < W; ++w) {
-                const int ce = (int)red_eq[e & 1][w], cg = (int)red_gt[e & 1][w];
-                if (w < warp) {
-                    eq_before += ce;
-                    gt_before += cg;
+            for (int d = 1; d < 32; d <<= 1) {
+                const unsigned te = __shfl_up_sync(0xffffffffu, ie, d), tg = __shfl_up_sync(0xffffffffu, ig, d);
+                if (lane >= d) {
+                    ie += te;
+                    ig += tg;
                 }
-                eq_seen += ce;
-                gt_seen += cg;
             }
-            const int eq_rank = eq_before + __popc(eq_ball & lt_mask);
-            const int gt_rank = gt_before + __popc(gt_ball & lt_mask);
+            if (lane < W) {
+                cnt_eq[warp][lane] = ie - ce;
+                cnt_gt[warp][lane] = ig - cg;
+            }
+            if (lane == 31) {
+                tot_eq[warp] = ie;
+                tot_gt[warp] = ig;
+            }
+        }
+        __syncthreads();
+        int eq_base = 0, gt_base = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const bool valid = (e * NT + (int)threadIdx.x) < nh;
+            const bool eq = valid && key[e] == T, gtk = valid && key[e] > T;
+            const unsigned eb = __ballot_sync(0xffffffffu, eq), gb = __ballot_sync(0xffffffffu, gtk);
+            const int eq_rank = eq_base + (int)cnt_eq[e][warp] + __popc(eb & lt_mask);
+            const int gt_rank = gt_base + (int)cnt_gt[e][warp] + __popc(gb & lt_mask);
             if (gtk || (eq && eq_rank < need)) {
                 const int pos = gt_rank + min(need, eq_rank);
                 idx[obase + pos] = e * NT + (int)threadIdx.x;
                 log_gate[obase + pos] = val[e] - lse;
             }
+            eq_base += (int)tot_eq[e];
+            gt_base += (int)tot_gt[e];
         }
     }
     for (int p = kk + (int)threadIdx.x; p < K; p += NT) {

@@ -18,8 +18,8 @@ is bracketed by barriers and the max over ranks is reported (weak scaling).
 Beside that headline line, after the timed steps (rank 0 prints them as extra
 keys of the same JSON line): the Qwen3-4B 8k and Qwen3-14B 2x32k layers
 (`configs`), the full-history variant (K >= #history) of the 32k layer with
-its dk/dv load balance (`full_history`), the fused stand-in scorer + select
-(`score_select`), and a decode scaling study over 64K-512K of context at batch
+its dk/dv load balance (`full_history`), the stand-in scorer + select in one
+call (`score_select`), and a decode scaling study over 64K-512K of context at batch
 1 and 8, sparse against the same kernel reading every block (`decode_scaling`,
 CUDA-graph replays). Every extra number is the median of CUDA-event times of
 back-to-back CUDA-graph replays (so short calls carry no host launch gaps; a
@@ -187,7 +187,7 @@ class ClockSampler:
     def start(self):
         try:
             cmd = ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
-                   "--format=csv,noheader,nounits", "-lms", "100"]
+                   "--format=csv,noheader,nounits", "-lms", "20"]
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -506,7 +506,7 @@ def run_extras(torch, sas, inputs, P, px, pc, dev, peaks, tpeak, a):
     out["full_history"] = {pc.name: fh}
     del ws, st
     torch.cuda.empty_cache()
-    # --- fused stand-in scorer + select on the headline workload (its scores are the stand-in)
+    # --- stand-in scorer + select on the headline workload (its scores are the stand-in)
     if "noise" in px:
         noise = px["noise"].to(dev)
         s_buf = torch.zeros_like(P["s"])
@@ -594,59 +594,92 @@ def decode_scaling(torch, sas, inputs, dev, peaks):
                                 "on other hardware, quoted as context only")
 
 
-def run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, world, dist, dev):
-    """Same step through the public API, inputs copied from pinned host memory
-    every step and every result read back to pinned host memory."""
-    hin_p = {k: px[k].pin_memory() for k in ("q", "k", "v", "do", "s")}
-    hin_d = {k: dx[k].pin_memory() for k in ("q", "s", "kv_len", "page_table")}
-    h2d = sum(t.numel() * t.element_size() for t in list(hin_p.values()) + list(hin_d.values()))
-    outs = {}
+def _pipelined(torch, hin, dsets, compute, steps, warmup, world, dist):
+    """Steps through the public API with host copies in the timed region.
 
-    def step(rec):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if rec else None
-        if rec:
-            ev[0].record()
-        for k, t in hin_p.items():
-            P[k].copy_(t, non_blocking=True)
-        sel = sas.select(P["s"], pc.K)
-        o, lse = sas.attn_fwd(P["q"], P["k"], P["v"], sel[0], sel[1], sel[2], sc_p)
-        dq, dk, dv, ds = sas.attn_bwd(P["q"], P["k"], P["v"], o, P["do"], lse, P["s"], sel[3], sel[0], sel[1],
-                                      sel[2], sc_p, workspace=ws_b)
-        res = dict(o=o, dq=dq, dk=dk, dv=dv, ds=ds)
-        for k, t in res.items():
-            if k not in outs:
-                outs[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-            outs[k].copy_(t, non_blocking=True)
-        if rec:
-            ev[1].record()
-        for k, t in hin_d.items():
-            Dd[k].copy_(t, non_blocking=True)
-        dsel = sas.select(Dd["s"], dc.K, kv_len=Dd["kv_len"])
-        od, _ = sas.decode_paged(Dd["q"], Dd["k_cache"], Dd["v_cache"], Dd["page_table"], Dd["kv_len"],
-                                 dsel[0], dsel[1], dsel[2], workspace=ws_d, with_lse=False)
-        if "od" not in outs:
-            outs["od"] = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
-        outs["od"].copy_(od, non_blocking=True)
-        if rec:
-            ev[2].record()
-        return ev
+    Step n copies its inputs (`hin`, pinned host tensors) into the device set
+    dsets[n % 2] on an input stream, runs compute(dset) -> {name: tensor} on the
+    current stream and copies every result into pinned host buffers on an
+    output stream, so the upload of step n + 1 and the download of step n - 1
+    overlap the compute of step n. A device set is rewritten only after the
+    compute that read it has finished. Returns the device time per step over
+    `steps` steps (CUDA events on the current stream, which waits for the other
+    two streams before the closing event) and the bytes read back per step."""
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    freed = [None, None]
+    outs = [{}, {}]
 
-    for _ in range(max(1, a.warmup)):
-        step(False)
+    def step(n):
+        b = dsets[n % 2]
+        if freed[n % 2] is not None:
+            s_in.wait_event(freed[n % 2])
+        with torch.cuda.stream(s_in):
+            for k, t in hin.items():
+                b[k].copy_(t, non_blocking=True)
+        comp.wait_stream(s_in)
+        res = compute(b)
+        freed[n % 2] = comp.record_event()
+        s_out.wait_stream(comp)
+        with torch.cuda.stream(s_out):
+            for k, t in res.items():
+                t.record_stream(s_out)
+                if k not in outs[n % 2]:
+                    outs[n % 2][k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                outs[n % 2][k].copy_(t, non_blocking=True)
+
+    for n in range(max(1, warmup)):
+        step(n)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    evs = [step(True) for _ in range(a.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    s_in.wait_stream(comp)
+    s_out.wait_stream(comp)
+    for n in range(steps):
+        step(n)
+    comp.wait_stream(s_in)
+    comp.wait_stream(s_out)
+    t1.record()
     torch.cuda.synchronize()
+    d2h = sum(t.numel() * t.element_size() for t in outs[0].values())
+    return t0.elapsed_time(t1) / steps, d2h
+
+
+def run_e2e(a, torch, sas, px, dx, P, Dd, pc, dc, sc_p, ws_b, ws_d, flops_fb, world, dist, dev):
+    """The prefill step and the decode step through the public API, each step's
+    inputs copied from pinned host memory and each step's results read back to
+    pinned host memory inside the timed region (pipelined over three streams)."""
+    hin_p = {k: px[k].pin_memory() for k in ("q", "k", "v", "do", "s")}
+    hin_d = {k: dx[k].pin_memory() for k in ("q", "s", "kv_len", "page_table")}
+    h2d_p = sum(t.numel() * t.element_size() for t in hin_p.values())
+    h2d_d = sum(t.numel() * t.element_size() for t in hin_d.values())
+
+    def prefill(b):
+        sel = sas.select(b["s"], pc.K)
+        o, lse = sas.attn_fwd(b["q"], b["k"], b["v"], sel[0], sel[1], sel[2], sc_p)
+        dq, dk, dv, ds = sas.attn_bwd(b["q"], b["k"], b["v"], o, b["do"], lse, b["s"], sel[3], sel[0], sel[1],
+                                      sel[2], sc_p, workspace=ws_b)
+        return dict(o=o, dq=dq, dk=dk, dv=dv, ds=ds)
+
+    def decode(b):
+        dsel = sas.select(b["s"], dc.K, kv_len=b["kv_len"])
+        od, _ = sas.decode_paged(b["q"], Dd["k_cache"], Dd["v_cache"], b["page_table"], b["kv_len"],
+                                 dsel[0], dsel[1], dsel[2], workspace=ws_d, with_lse=False)
+        return dict(od=od)
+
+    sets_p = [{k: P[k] for k in hin_p}, {k: torch.empty_like(P[k]) for k in hin_p}]
+    sets_d = [{k: Dd[k] for k in hin_d}, {k: torch.empty_like(Dd[k]) for k in hin_d}]
+    pre, d2h_p = _pipelined(torch, hin_p, sets_p, prefill, a.steps, a.warmup, world, dist)
+    dec, d2h_d = _pipelined(torch, hin_d, sets_d, decode, a.steps, a.warmup, world, dist)
     sas.get_error_flag()
-    pre = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
-    dec = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
     pre, dec = max_over_ranks([pre, dec], dist, dev)
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
     return dict(value=round(weak_tflops(world, flops_fb, pre), 3), unit="TFLOPS",
-                h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
+                h2d_bytes_per_step=int(h2d_p + h2d_d), d2h_bytes_per_step=int(d2h_p + d2h_d),
                 ms_prefill=round(pre, 3), ms_decode=round(dec, 3),
-                decode_tokens_per_s=round(world * dc.N / (dec * 1e-3), 1))
+                decode_tokens_per_s=round(world * dc.N / (dec * 1e-3), 1),
+                overlap="upload of step n+1 and download of step n-1 run beside step n's kernels")
 
 
 # ---------------------------------------------------------------------------

@@ -221,8 +221,8 @@ sas_status sas_attn_bwd_varlen(sas_dtype dtype, const void *q, const void *k, co
 size_t sas_score_select_workspace_size(int B, int S, int Hq, int Hkv, int D);
 
 /*
- * sas_score_select - block-pooled stand-in selector scores, fused with the
- * Top-K selection and the log-gates of sas_select (prefill).
+ * sas_score_select - block-pooled stand-in selector scores, followed in the
+ * same call by the Top-K selection and the log-gates of sas_select (prefill).
  * SAS review §2.2: the selector scores each history block of a query block,
  * s = R_theta(q, {K_Bm}), and the Top-K are kept; §2.4, eq. log g. The
  * trained selector (AttnGate) is not part of this library; its stand-in is

@@ -1,4 +1,4 @@
-"""The fused stand-in scorer + select (sas_score_select) through the C ABI against the
+"""The stand-in scorer + select (sas_score_select) through the C ABI against the
 oracle's fp64 stand-in scores (oracle.standin_scores) and Top-K (oracle.select).
 
 The GPU sums the bf16 inputs in fp32, so its scores differ from the fp64 oracle's by

@@ -1,5 +1,5 @@
-// sas_score_select: block-pooled stand-in selector scores fused with the
-// Top-K selection and the log-gates.
+// sas_score_select: block-pooled stand-in selector scores, then the Top-K
+// selection and the log-gates.
 //
 // SAS review (paper.oopus.info) §2.2: the selector scores every history block
 // of a query block, s = R_theta(q, {K_Bm}), and the Top-K are kept; §2.4, eq.
@@ -9,22 +9,16 @@
 //              . mean_{64 rows of block j}(k[h]) / sqrt(D)  (+ noise[b,h,i,j]),
 // for j < i, the noise being an optional input.
 //
-// Two kernels:
+// Prefill, three kernels:
 //  * pool_kernel - one CTA per (query block, batch): sums the 64 rows of q
 //    (all query heads) and of k in fp32 with 16-byte loads, then folds the G
 //    heads of each KV head; writes the block means qp, kp [B, Hkv, NQB, D]
 //    (fp32, in the workspace). Reads q and k once: HBM-bound.
-//  * score_select_kernel - one warp per selection row (b, h, i), eight rows of
-//    one (b, h) per CTA. Chunks of 32 pooled keys are staged in shared memory
-//    (one row per lane, 16-byte rows padded against bank conflicts, read as
-//    float4) and every lane forms
-//    the dot product of its key with the warp's pooled query, so that lane l
-//    holds s[i][32 e + l] - the register layout of the warp-row selection,
-//    which runs next (select_row.cuh). s is written once (the backward's
-//    Jacobian reads it).
-// Rows of more than 512 history blocks: the scores are written by the same
-// kernel without the selection, then selected by sas_select's CTA-per-row
-// kernel.
+//  * score_tile_kernel - the lower triangle of qp kp^T / sqrt(D) (+ noise) in
+//    64 x 64 tiles, 4 x 4 products per thread from shared memory; s is
+//    written once (the backward's Jacobian reads it).
+//  * the selection of sas_select on those rows (warp per row, CTA per row
+//    beyond 512 history blocks), reading s back from L2.
 //
 // Decode (sas_pool_pages, sas_score_select_decode): the mean key of every
 // (page, KV head) is kept in a pooled-key cache (fp32 [pages, Hkv, D]),
@@ -35,150 +29,144 @@
 // pooled over its GQA group; the scores go to sas_select's decode path.
 #include "common.cuh"
 #include "launch.h"
-#include "select_row.cuh"
 
 namespace sas {
 namespace {
 
 constexpr int kPoolThreads = 256;
-constexpr int kRowsPerCta = 8;
 
 // qp[b, h, i, :] = mean over the 64 rows of block i and the G query heads of
 // KV head h; kp[b, h, i, :] = mean over the 64 rows of block i of k[:, :, h].
-__global__ void __launch_bounds__(kPoolThreads)
+// One CTA per (query block i, KV head h, batch b): a token row of the group
+// is C = (G + 1) D / 8 16-byte chunks (G query heads, contiguous in q, then
+// the KV head's key row), thread t sums chunk t % C over the rows
+// t / C, t / C + R, ... (R = 256 / C row groups), the R partial sums meet in
+// shared memory and D threads fold them and the G heads. Small CTAs keep
+// every SM's share of the bytes within one CTA of the mean.
+__global__ void __launch_bounds__(kPoolThreads, 4)     // eight 16-byte loads in flight per thread
 pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int S, int Hq, int Hkv, int D,
             float* __restrict__ qp, float* __restrict__ kp) {
-    extern __shared__ float acc[];                  // [Hq * D] q sums, then [Hkv * D] k sums
-    const int i = blockIdx.x, b = blockIdx.y, NQB = gridDim.x;
+    extern __shared__ float acc[];                  // [R][C * 8] partial sums
+    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z, NQB = gridDim.x;
     const int G = Hq / Hkv;
+    const int cq = G * D / 8, C = cq + D / 8;       // chunks of the group's q row, of the whole row
+    const int R = max(1, kPoolThreads / C);
     const long long row0 = (long long)b * S + (long long)i * kBlock;
-    for (int pass = 0; pass < 2; ++pass) {
-        const __nv_bfloat16* src = pass == 0 ? q : k;
-        const int cols = (pass == 0 ? Hq : Hkv) * D;             // bf16 per token row
-        float* dst = acc + (pass == 0 ? 0 : Hq * D);
-        for (int c = threadIdx.x; c < cols / 8; c += kPoolThreads) {   // 16-byte chunk c of every row
-            float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            const uint4* p = reinterpret_cast<const uint4*>(src + row0 * cols) + c;
+    const uint4* qsrc = reinterpret_cast<const uint4*>(q + (row0 * Hq + (long long)h * G) * D);
+    const uint4* ksrc = reinterpret_cast<const uint4*>(k + (row0 * Hkv + h) * D);
+    const long long qstride = (long long)Hq * D / 8, kstride = (long long)Hkv * D / 8;   // chunks per token row
+    for (int u = threadIdx.x; u < C * R; u += kPoolThreads) {
+        const int c = u % C, rg = u / C;
+        const uint4* p = c < cq ? qsrc + c : ksrc + (c - cq);
+        const long long stride = c < cq ? qstride : kstride;
+        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-            for (int r = 0; r < kBlock; ++r) {
-                const uint4 w = __ldg(p + (long long)r * (cols / 8));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int r = rg; r < kBlock; r += R) {
+            const uint4 w = __ldg(p + (long long)r * stride);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = bf16x2_to_f32(ws[e]);
-                    a[2 * e] += f.x;
-                    a[2 * e + 1] += f.y;
-                }
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = bf16x2_to_f32(ws[e]);
+                a[2 * e] += f.x;
+                a[2 * e + 1] += f.y;
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dst[c * 8 + e] = a[e];
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[(size_t)rg * C * 8 + c * 8 + e] = a[e];
     }
     __syncthreads();
     const float inv_q = 1.f / (float)(kBlock * G), inv_k = 1.f / (float)kBlock;
-    for (int t = threadIdx.x; t < Hkv * D; t += kPoolThreads) {
-        const int h = t / D, d = t % D;
-        float sq = 0.f;
-        for (int g = 0; g < G; ++g) sq += acc[(h * G + g) * D + d];
+    for (int d = threadIdx.x; d < D; d += kPoolThreads) {
+        float sq = 0.f, sk = 0.f;
+        for (int rg = 0; rg < R; ++rg) {
+            const float* pr = acc + (size_t)rg * C * 8;
+            for (int g = 0; g < G; ++g) sq += pr[g * D + d];
+            sk += pr[G * D + d];
+        }
         const long long o = (((long long)b * Hkv + h) * NQB + i) * D + d;
         qp[o] = sq * inv_q;
-        kp[o] = acc[Hq * D + t] * inv_k;
+        kp[o] = sk * inv_k;
     }
 }
 
-// Scores of the rows of one CTA: warp w owns row i = 8 blockIdx.x + w of
-// (b, h) = blockIdx.y; lane l of the warp computes j = 32 e + l for every
-// chunk e below `chunks`. The pooled keys of chunk e are staged by the CTA.
-template <int E, bool kSelect>
-__global__ void __launch_bounds__(kRowsPerCta * 32, 3)     // three CTAs per SM: 85 registers at most
-score_select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int NQB, int D, float inv_sqrt_d,
-                    const float* __restrict__ noise, int ld_noise, float* __restrict__ s, int ld_s, int K,
-                    int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ log_gate,
-                    float* __restrict__ lse_s, int* status) {
-    extern __shared__ float sm[];
-    // two [32][D + 4] buffers of pooled keys (chunk e in buffer e & 1): rows 16-byte aligned,
-    // and the +4 padding keeps the eight lanes of each quarter-warp 128-bit load on distinct
-    // banks. Chunk e + 1 is loaded into registers while chunk e is used.
-    const int ldk = D + 4;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* qrow = sm + 2 * 32 * ldk + warp * D;                // this warp's pooled query
+// Scores of one 64 x 64 tile (query blocks [64 ti, 64 ti + 64) x key blocks
+// [64 tj, 64 tj + 64), tj <= ti) of (b, h) = blockIdx.y: the tile's pooled
+// queries and keys are staged in shared memory transposed ([d][row], rows
+// padded to 68 floats), and each thread accumulates a 4 x 4 block of dot
+// products over D from two 128-bit loads per d (the query load is a
+// broadcast, the key loads of a half-warp cover 256 contiguous bytes), so
+// every staged value feeds 4 products. Entries with j < i get noise added and
+// are written; the selection then reads them back (from L2).
+constexpr int kTile = 64;
+constexpr int kTileLd = kTile + 4;
+__global__ void __launch_bounds__(256)
+score_tile_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int NQB, int D, float inv_sqrt_d,
+                  const float* __restrict__ noise, int ld_noise, float* __restrict__ s, int ld_s) {
+    extern __shared__ __align__(16) float sm[];
+    float* qs = sm;                                   // [D][kTileLd] pooled queries of the tile's rows
+    float* ks = sm + (size_t)D * kTileLd;             // [D][kTileLd] pooled keys of the tile's columns
+    // lower-triangle tile index -> (ti, tj): tiles of row ti are ti*(ti+1)/2 .. + ti
+    const int t = blockIdx.x;
+    int ti = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+    while (ti * (ti + 1) / 2 > t) --ti;
+    const int tj = t - ti * (ti + 1) / 2;
     const long long bh = blockIdx.y;
-    const int i = blockIdx.x * kRowsPerCta + warp;
-    const bool live = i < NQB;
-    const int i_max = min(NQB - 1, (int)blockIdx.x * kRowsPerCta + kRowsPerCta - 1);   // longest row of the CTA
-    const long long row = bh * NQB + i;
-    if (live)
-        for (int d = lane; d < D; d += 32) qrow[d] = qp[row * D + d];
-    const int chunks = kSelect ? E : (i_max + 31) / 32;
-    const int used = (i_max + 31) / 32;                        // chunks holding some j < i_max
-    constexpr int kPer = 32 * 128 / 4 / (kRowsPerCta * 32);    // float4 of a chunk per thread (D = 128)
-    float4 nxt[kPer];
-    auto fetch = [&](int e) {                                  // chunk e -> registers
+    const int i0 = ti * kTile, j0 = tj * kTile;
+    // lanes of a warp take consecutive rows: 16-byte global loads, conflict-free transposed stores;
+    // eight loads of each operand are in flight per thread before the stores
+    constexpr int kU = 8;
+    const int units = kTile * (D / 4);
+    for (int e0 = threadIdx.x; e0 < units; e0 += kU * blockDim.x) {
+        float4 qv[kU], kv[kU];
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int t = threadIdx.x + u * kRowsPerCta * 32;
-            const int r = t / (D / 4), d4 = t % (D / 4);
-            nxt[u] = (t < 8 * D && e * 32 + r < i_max)
-                         ? reinterpret_cast<const float4*>(kp + (bh * NQB + e * 32 + r) * D)[d4]
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * blockDim.x;
+            const int r = e % kTile, d4 = e / kTile;
+            const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+            const bool in = e < units;
+            qv[u] = (in && i0 + r < NQB) ? reinterpret_cast<const float4*>(qp + (bh * NQB + i0 + r) * D)[d4] : zero;
+            kv[u] = (in && j0 + r < NQB) ? reinterpret_cast<const float4*>(kp + (bh * NQB + j0 + r) * D)[d4] : zero;
         }
-    };
-    auto stash = [&](int e) {                                  // registers -> buffer e & 1
-        float* kc = sm + (e & 1) * 32 * ldk;
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int t = threadIdx.x + u * kRowsPerCta * 32;
-            if (t < 8 * D) reinterpret_cast<float4*>(kc + (t / (D / 4)) * ldk)[t % (D / 4)] = nxt[u];
+        for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * blockDim.x;
+            if (e >= units) break;
+            const int r = e % kTile, d4 = e / kTile;
+            float* qd = qs + (4 * d4) * kTileLd + r;
+            float* kd = ks + (4 * d4) * kTileLd + r;
+            qd[0] = qv[u].x; qd[kTileLd] = qv[u].y; qd[2 * kTileLd] = qv[u].z; qd[3 * kTileLd] = qv[u].w;
+            kd[0] = kv[u].x; kd[kTileLd] = kv[u].y; kd[2 * kTileLd] = kv[u].z; kd[3 * kTileLd] = kv[u].w;
         }
-    };
-    float val[kSelect ? E : 1];
-#pragma unroll
-    for (int e = 0; e < (kSelect ? E : 1); ++e) val[e] = -INFINITY;
-    if (used > 0) {
-        fetch(0);
-        stash(0);
     }
-    for (int e = 0; e < chunks; ++e) {
-        if (e < used) {                                        // the same for the whole CTA
-            if (e + 1 < used) fetch(e + 1);                    // in flight while chunk e is used
-            __syncthreads();                                   // chunk e is in its buffer
-        }
-        const int j = e * 32 + lane;
-        if (live && j < i) {
-            const float4* kr = reinterpret_cast<const float4*>(sm + (e & 1) * 32 * ldk + lane * ldk);
-            const float4* qr = reinterpret_cast<const float4*>(qrow);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;       // four chains
-            for (int d4 = 0; d4 < D / 4; ++d4) {
-                const float4 kv = kr[d4], qv = qr[d4];
-                a0 = fmaf(qv.x, kv.x, a0);
-                a1 = fmaf(qv.y, kv.y, a1);
-                a2 = fmaf(qv.z, kv.z, a2);
-                a3 = fmaf(qv.w, kv.w, a3);
-            }
-            float v = ((a0 + a1) + (a2 + a3)) * inv_sqrt_d;
-            if (noise != nullptr) v += __ldg(noise + row * (long long)ld_noise + j);
-            s[row * (long long)ld_s + j] = v;
-            if (kSelect) {
+    __syncthreads();
+    const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+    float acc[4][4] = {};
+#pragma unroll 2
+    for (int d = 0; d < D; ++d) {
+        const float4 av = *reinterpret_cast<const float4*>(qs + d * kTileLd + ty * 4);
+        const float4 cv = *reinterpret_cast<const float4*>(ks + d * kTileLd + tx * 4);
+        const float a[4] = {av.x, av.y, av.z, av.w}, c[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-                for (int ee = 0; ee < (kSelect ? E : 1); ++ee)
-                    if (ee == e) val[ee] = v;
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], c[w], acc[u][w]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = i0 + ty * 4 + u;
+        if (i >= NQB) continue;
+        const long long row = bh * NQB + i;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int j = j0 + tx * 4 + w;
+            if (j < i) {
+                float v = acc[u][w] * inv_sqrt_d;
+                if (noise != nullptr) v += __ldg(noise + row * (long long)ld_noise + j);
+                s[row * (long long)ld_s + j] = v;
             }
         }
-        if (e + 1 < used) stash(e + 1);                        // the other buffer: no one reads it now
     }
-    if (kSelect && live) select_warp_row<kSelect ? E : 1>(val, i, K, row, idx, cnt, log_gate, lse_s, status);
-}
-
-template <int E>
-cudaError_t go_fused(const float* qp, const float* kp, int B, int Hkv, int NQB, int D, float inv, const float* noise,
-                     int ld_noise, float* s, int ld_s, int K, int32_t* idx, int32_t* cnt, float* lg, float* lse_s,
-                     int* status, cudaStream_t st) {
-    const dim3 grid((NQB + kRowsPerCta - 1) / kRowsPerCta, B * Hkv);
-    const size_t sm = sizeof(float) * (2 * 32 * (D + 4) + kRowsPerCta * D);
-    score_select_kernel<E, true><<<grid, kRowsPerCta * 32, sm, st>>>(qp, kp, NQB, D, inv, noise, ld_noise, s, ld_s,
-                                                                     K, idx, cnt, lg, lse_s, status);
-    count_launches(1);
-    return cudaGetLastError();
 }
 
 // kpool[page, h, :] = mean over the 64 rows of k_cache[page, h] (fp32 sums).
@@ -228,7 +216,7 @@ pool_pages_kernel(const __nv_bfloat16* __restrict__ k_cache, int num_pages, int 
 // [128 chunk, 128 chunk + 128) of row (n, h); warp w takes 4 blocks per round,
 // 8 lanes per block, each lane a strided quarter (D = 128) of the pooled key.
 constexpr int kDecScoreBlocks = 128;
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 score_decode_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ kpool, int num_pages,
                     const int32_t* __restrict__ page_table, int max_pages, const int32_t* __restrict__ kv_len,
                     int Hq, int Hkv, int D, float inv_sqrt_d, const float* __restrict__ noise, int ld_noise,
@@ -314,31 +302,25 @@ cudaError_t launch_score_select(const ScoreArgs& a, cudaStream_t st) {
     const size_t n = (size_t)a.B * a.Hkv * NQB * a.D;
     float* qp = static_cast<float*>(a.workspace);
     float* kp = qp + (((sizeof(float) * n + 255) & ~size_t(255)) / sizeof(float));
-    const size_t psm = sizeof(float) * (size_t)(a.Hq + a.Hkv) * a.D;
+    const int C = (a.Hq / a.Hkv + 1) * a.D / 8;
+    const size_t psm = sizeof(float) * 8 * (size_t)C * (size_t)std::max(1, kPoolThreads / C);
     cudaError_t e = cudaFuncSetAttribute(pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
     if (e != cudaSuccess) return e;
-    pool_kernel<<<dim3(NQB, a.B), kPoolThreads, psm, st>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k,
-                                                             a.S, a.Hq, a.Hkv, a.D, qp, kp);
+    pool_kernel<<<dim3(NQB, a.Hkv, a.B), kPoolThreads, psm, st>>>((const __nv_bfloat16*)a.q,
+                                                                    (const __nv_bfloat16*)a.k, a.S, a.Hq, a.Hkv,
+                                                                    a.D, qp, kp);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const float inv = 1.f / sqrtf((float)a.D);
-    const int max_hist = NQB - 1;
-#define SAS_FUSED_ARGS qp, kp, a.B, a.Hkv, NQB, a.D, inv, a.noise, a.ld_noise, a.s, a.ld_s, a.K, a.idx, a.cnt, \
-                       a.log_gate, a.lse_s, a.status, st
-    if (max_hist <= 32) return go_fused<1>(SAS_FUSED_ARGS);
-    if (max_hist <= 64) return go_fused<2>(SAS_FUSED_ARGS);
-    if (max_hist <= 128) return go_fused<4>(SAS_FUSED_ARGS);
-    if (max_hist <= 256) return go_fused<8>(SAS_FUSED_ARGS);
-    if (max_hist <= 512) return go_fused<16>(SAS_FUSED_ARGS);
-#undef SAS_FUSED_ARGS
-    // longer rows: scores first, then the CTA-per-row selection
-    const dim3 grid((NQB + kRowsPerCta - 1) / kRowsPerCta, a.B * a.Hkv);
-    const size_t sm = sizeof(float) * (2 * 32 * (a.D + 4) + kRowsPerCta * a.D);
-    score_select_kernel<1, false><<<grid, kRowsPerCta * 32, sm, st>>>(
-        qp, kp, NQB, a.D, inv, a.noise, a.ld_noise, a.s, a.ld_s, a.K, a.idx, a.cnt, a.log_gate, a.lse_s, a.status);
+    const int nt = (NQB + kTile - 1) / kTile;
+    const size_t tsm = sizeof(float) * 2 * (size_t)a.D * kTileLd;
+    if ((e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm)) !=
+        cudaSuccess)
+        return e;
+    score_tile_kernel<<<dim3(nt * (nt + 1) / 2, a.B * a.Hkv), 256, tsm, st>>>(
+        qp, kp, NQB, a.D, 1.f / sqrtf((float)a.D), a.noise, a.ld_noise, a.s, a.ld_s);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return launch_select(a.s, a.B, a.Hkv, NQB, a.ld_s, nullptr, nullptr, a.K, max_hist, a.idx, a.cnt, a.log_gate,
+    return launch_select(a.s, a.B, a.Hkv, NQB, a.ld_s, nullptr, nullptr, a.K, NQB - 1, a.idx, a.cnt, a.log_gate,
                          a.lse_s, a.status, st);
 }
 

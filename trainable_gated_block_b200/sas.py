@@ -160,8 +160,8 @@ def select_varlen(s, K: int, cu_seqlens, block_size: int = 64):
 
 
 def score_select(q, k, K: int, noise=None, block_size: int = 64, workspace=None, s_out=None):
-    """Stand-in selector scores (block-pooled q . k / sqrt(D) + noise) fused with Top-K and
-    log-gates. q [B,S,Hq,D], k [B,S,Hkv,D] bf16; noise [B,Hkv,NQB,ld] fp32 or None.
+    """Stand-in selector scores (block-pooled q . k / sqrt(D) + noise), then Top-K and
+    log-gates, in one call. q [B,S,Hq,D], k [B,S,Hkv,D] bf16; noise [B,Hkv,NQB,ld] fp32 or None.
     Returns s [B,Hkv,NQB,NQB] (entries j >= i are whatever s_out held, zero when it is
     allocated here), idx, cnt, log_gate, lse_s."""
     _contig(q, k, noise)

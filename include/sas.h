@@ -240,6 +240,8 @@ size_t sas_score_select_workspace_size(int B, int S, int Hq, int Hkv, int D);
  * idx, cnt, log_gate, lse_s   as sas_select writes them for these scores.
  * workspace device, 256-byte aligned, ws_bytes >= sas_score_select_workspace_size
  *          (it holds the pooled queries and keys).
+ * SAS_ERR_UNSUPPORTED for rows of more than 16384 history blocks, for
+ * B * Hkv > 65535, and when (Hq + Hkv) * D fp32 values exceed 200 KiB.
  */
 sas_status sas_score_select(const void *q, const void *k, const float *noise, int ld_noise,
                             int B, int S, int Hq, int Hkv, int D, int block_size, int K,

@@ -123,3 +123,26 @@ def test_varlen_rejects_bad_arguments(L):
     r = b(sas.SAS_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None,
           3, 100, 250, 4, 2, 128, 64, 2, 0.1, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0x10000), 1 << 30, None)
     assert r == sas.SAS_ERR_INVALID_ARG
+
+
+def test_score_select_rejects_bad_arguments(L):
+    f = L.sas_score_select
+    ws = ctypes.c_void_p(0x10000)
+    #       q     k     noise ld  B  S    Hq Hkv D   bs  K  s     ld_s idx   cnt   lg    lse_s ws  bytes    stream
+    args = [FAKE, FAKE, None, 0, 1, 512, 8, 2, 128, 64, 2, FAKE, 8, FAKE, FAKE, FAKE, FAKE, ws, 1 << 30, None]
+    bad = list(args); bad[0] = None                         # no q
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[5] = 500                          # S not a multiple of 64
+    assert f(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[8] = 96                           # D
+    assert f(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[12] = 7                           # ld_s below the 8 blocks
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[5] = 64 * 16386; bad[12] = 16386  # 16385 history blocks
+    assert f(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[4] = 32768; bad[5] = 64; bad[12] = 1   # B * Hkv above a grid dimension
+    assert f(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[17] = ctypes.c_void_p(0x10010)    # workspace alignment
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[18] = 16                          # workspace too small
+    assert f(*bad) == sas.SAS_ERR_INVALID_ARG

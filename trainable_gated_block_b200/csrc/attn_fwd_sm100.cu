@@ -380,30 +380,66 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 tmem_ld32(tT + 64 * buf, raw[0]);
                 tmem_ld32(tT + 64 * buf + 32, raw[1]);
                 tmem_wait_ld();
-                float x[64];
+                // logit (log2 units) = S * scale2 + bias2. On a block without masked
+                // keys the row max is taken over the raw S (the affine map is monotonic,
+                // so the maximum is the same number) and each P costs one FMA and one
+                // exp2; on the diagonal or a flagged block the masked logits replace S
+                // in place and the same FMA runs with scale 1.
+                const bool masked = m.cur || !m.live;
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // 4 independent chains
-                if (m.cur || !m.live) {
+                float mx, sc, bias;
+                if (masked) {
 #pragma unroll
                     for (int u = 0; u < 64; ++u) {
                         const bool live = m.live && u <= r_in;
-                        x[u] = live ? fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2) : -INFINITY;
-                        mx4[u & 3] = fmaxf(mx4[u & 3], x[u]);
+                        const float x = live ? fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2) : -INFINITY;
+                        raw[u >> 5][u & 31] = __float_as_uint(x);
+                        mx4[u & 3] = fmaxf(mx4[u & 3], x);
                     }
+                    mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                    sc = 1.f;
+                    bias = 0.f;
                 } else {
+                    float r;                             // the S that gives the largest logit
+                    if (p.scale2 >= 0.f) {
 #pragma unroll
-                    for (int u = 0; u < 64; ++u) {
-                        x[u] = fmaf(__uint_as_float(raw[u >> 5][u & 31]), p.scale2, m.bias2);
-                        mx4[u & 3] = fmaxf(mx4[u & 3], x[u]);
+                        for (int u = 0; u < 64; ++u) mx4[u & 3] = fmaxf(mx4[u & 3], __uint_as_float(raw[u >> 5][u & 31]));
+                        r = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                    } else {
+                        float mn4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+#pragma unroll
+                        for (int u = 0; u < 64; ++u) mn4[u & 3] = fminf(mn4[u & 3], __uint_as_float(raw[u >> 5][u & 31]));
+                        r = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
                     }
+                    mx = fmaf(r, p.scale2, m.bias2);
+                    sc = p.scale2;
+                    bias = m.bias2;
                 }
-                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 const float m_new = fmaxf(m_ref, mx);
                 const bool need = m_new > m_ref + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need) && k > 0) {
+                const bool rescale = __any_sync(0xffffffffu, need) && k > 0;    // warp-uniform
+                const float f = need ? exp2f(m_ref - m_new) : 1.f;                // O and l scale
+                if (need) {
+                    l *= f;
+                    m_ref = m_new;
+                }
+                const float c = bias - ((m_ref == -INFINITY) ? 0.f : m_ref);   // P = 2^(S sc + c)
+                uint32_t pk[32];
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};     // 4 independent chains
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int u = 2 * e;
+                    const float p0 = fast_exp2(fmaf(__uint_as_float(raw[u >> 5][u & 31]), sc, c));
+                    const float p1 = fast_exp2(fmaf(__uint_as_float(raw[(u + 1) >> 5][(u + 1) & 31]), sc, c));
+                    l4[e & 3] += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                tmem_st32(tT + 64 * buf, pk);
+                if (rescale) {
                     // O is rescaled in TMEM: PV of the previous step must be complete
                     if (!(ok = wait_count(&bars->pv_count[t], pv_it + k, abort, p.status))) break;
                     tc_fence_after();
-                    const float f = need ? exp2f(m_ref - m_new) : 1.f;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         uint32_t ov[32];
@@ -414,22 +450,6 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         tmem_st32(tO + q4 * 32, ov);
                     }
                 }
-                if (need) {
-                    l *= exp2f(m_ref - m_new);
-                    m_ref = m_new;
-                }
-                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                uint32_t pk[32];
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};     // 4 independent chains
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = fast_exp2(x[2 * e] - m_use);
-                    const float p1 = fast_exp2(x[2 * e + 1] - m_use);
-                    l4[e & 3] += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
-                }
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-                tmem_st32(tT + 64 * buf, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars->p_full[t][buf]);

@@ -323,6 +323,8 @@ sas_status sas_score_select(const void* q, const void* k, const float* noise, in
         return fail(SAS_ERR_INVALID_ARG, "%s: row strides (ld_s=%d, ld_noise=%d) below %d blocks", fn, ld_s, ld_noise, nqb);
     if (nqb - 1 > kMaxHistory)
         return fail(SAS_ERR_UNSUPPORTED, "%s: rows of more than %d history blocks", fn, kMaxHistory);
+    if ((long long)B * Hkv > 65535)     // grid dimension of the score tiles
+        return fail(SAS_ERR_UNSUPPORTED, "%s: B*Hkv=%lld above 65535", fn, (long long)B * Hkv);
     if ((size_t)(Hq + Hkv) * D * sizeof(float) > 200 * 1024)
         return fail(SAS_ERR_UNSUPPORTED, "%s: %d + %d heads of %d dims exceed the pooling CTA's shared memory", fn,
                     Hq, Hkv, D);

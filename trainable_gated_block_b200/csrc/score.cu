@@ -37,7 +37,8 @@ constexpr int kPoolThreads = 256;
 
 // qp[b, h, i, :] = mean over the 64 rows of block i and the G query heads of
 // KV head h; kp[b, h, i, :] = mean over the 64 rows of block i of k[:, :, h].
-// One CTA per (query block i, KV head h, batch b): a token row of the group
+// One CTA per (KV head h, query block i, batch b), h fastest so that the CTAs
+// running together read whole token rows of q and k: a token row of the group
 // is C = (G + 1) D / 8 16-byte chunks (G query heads, contiguous in q, then
 // the KV head's key row), thread t sums chunk t % C over the rows
 // t / C, t / C + R, ... (R = 256 / C row groups), the R partial sums meet in
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(kPoolThreads, 4)     // eight 16-byte loads in
 pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int S, int Hq, int Hkv, int D,
             float* __restrict__ qp, float* __restrict__ kp) {
     extern __shared__ float acc[];                  // [R][C * 8] partial sums
-    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z, NQB = gridDim.x;
+    const int h = blockIdx.x, i = blockIdx.y, b = blockIdx.z, NQB = gridDim.y;
     const int G = Hq / Hkv;
     const int cq = G * D / 8, C = cq + D / 8;       // chunks of the group's q row, of the whole row
     const int R = max(1, kPoolThreads / C);
@@ -306,7 +307,7 @@ cudaError_t launch_score_select(const ScoreArgs& a, cudaStream_t st) {
     const size_t psm = sizeof(float) * 8 * (size_t)C * (size_t)std::max(1, kPoolThreads / C);
     cudaError_t e = cudaFuncSetAttribute(pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
     if (e != cudaSuccess) return e;
-    pool_kernel<<<dim3(NQB, a.Hkv, a.B), kPoolThreads, psm, st>>>((const __nv_bfloat16*)a.q,
+    pool_kernel<<<dim3(a.Hkv, NQB, a.B), kPoolThreads, psm, st>>>((const __nv_bfloat16*)a.q,
                                                                     (const __nv_bfloat16*)a.k, a.S, a.Hq, a.Hkv,
                                                                     a.D, qp, kp);
     count_launches(1);

@@ -1,5 +1,5 @@
-// Top-K selection and log-gates of one score row held by one warp (shared by
-// sas_select and the fused stand-in scorer).
+// Top-K selection and log-gates of one score row held by one warp (the
+// warp-per-row kernel of sas_select).
 //
 // SAS review (paper.oopus.info) §2.2 (Top-K of the selector scores) and §2.4,
 // eq. log g (log g_m = s_m - LSE(s) over all history blocks). Exact and

@@ -124,6 +124,13 @@ SMALL = [
     ("bf16-S1000-g5", "bf16", 1, 1000, 10, 2, 128, 4, 2.0),
     ("bf16-S65-d64", "bf16", 1, 65, 4, 2, 64, 2, 1.0),
     ("bf16-S1", "bf16", 2, 1, 8, 2, 128, 2, 1.0),
+    # other GQA group sizes on the tensor-core path: one head per KV head (a
+    # padding head in every tile), two (one tile per group), three (one tile
+    # and a half-padded one) and eight (two tiles in each of two groups)
+    ("bf16-g1", "bf16", 1, 576, 2, 2, 128, 3, 1.0),
+    ("bf16-g2", "bf16", 2, 448, 4, 2, 128, 2, 1.0),
+    ("bf16-g3-S300", "bf16", 1, 300, 6, 2, 128, 2, 1.0),
+    ("bf16-g8", "bf16", 1, 640, 8, 1, 128, 4, 1.0),
 ]
 
 

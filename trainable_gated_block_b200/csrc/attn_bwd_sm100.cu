@@ -93,30 +93,35 @@ template <bool kMask>
 __device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32_t (&pv)[32], int hf, float scale2,
                                           float off, float sm_scale, float drs, int lim, uint8_t* bufP,
                                           uint8_t* bufS, int row) {
-    float gs4[4] = {0.f, 0.f, 0.f, 0.f};          // 4 independent chains
+    // two keys per f32x2 instruction (same rounding per key as the scalar forms)
+    const unsigned long long sc2 = f2_pack(scale2, scale2), off2 = f2_pack(off, off);
+    const unsigned long long sm2 = f2_pack(sm_scale, sm_scale), nd2 = f2_pack(-drs, -drs);
+    unsigned long long gs2[2] = {0ull, 0ull};       // 2 independent chains of pairs
 #pragma unroll
     for (int c = 0; c < 4; ++c) {                 // 16-byte chunk = keys 8c .. 8c+7 of the half
         uint32_t pp[4], dd[4];
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
-            float pr[2], ds[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int e = 8 * c + 2 * e2 + q;
-                float x = fmaf(__uint_as_float(sv[e]), scale2, off);
-                if (kMask) x = (32 * hf + e > lim) ? -INFINITY : x;
-                pr[q] = fast_exp2(x);
-                ds[q] = pr[q] * fmaf(__uint_as_float(pv[e]), sm_scale, -drs);
-                gs4[e2] += ds[q];
+            const int e = 8 * c + 2 * e2;
+            float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, off2));
+            if (kMask) {
+                x.x = (32 * hf + e > lim) ? -INFINITY : x.x;
+                x.y = (32 * hf + e + 1 > lim) ? -INFINITY : x.y;
             }
-            pp[e2] = pack_bf16x2(pr[0], pr[1]);
-            dd[e2] = pack_bf16x2(ds[0], ds[1]);
+            const float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
+            const unsigned long long dp = f2_fma(f2_pack(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])), sm2, nd2);
+            const unsigned long long ds = f2_mul(f2_pack(p0, p1), dp);
+            gs2[e2 & 1] = f2_add(gs2[e2 & 1], ds);
+            const float2 d = f2_unpack(ds);
+            pp[e2] = pack_bf16x2(p0, p1);
+            dd[e2] = pack_bf16x2(d.x, d.y);
         }
         const int ch = 4 * hf + c;
         if (bufP) *reinterpret_cast<uint4*>(bufP + sw128_offset(row, ch)) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
         *reinterpret_cast<uint4*>(bufS + sw128_offset(row, ch)) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
     }
-    return (gs4[0] + gs4[1]) + (gs4[2] + gs4[3]);
+    const float2 g = f2_unpack(f2_add(gs2[0], gs2[1]));
+    return g.x + g.y;
 }
 
 // ===================================================================== dq

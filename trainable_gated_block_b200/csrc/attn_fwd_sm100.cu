@@ -403,7 +403,9 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     float r;                             // the S that gives the largest logit
                     if (p.scale2 >= 0.f) {
 #pragma unroll
-                        for (int u = 0; u < 64; ++u) mx4[u & 3] = fmaxf(mx4[u & 3], __uint_as_float(raw[u >> 5][u & 31]));
+                        for (int u = 0; u < 64; u += 2)     // two keys per three-input max
+                            mx4[(u >> 1) & 3] = max3(mx4[(u >> 1) & 3], __uint_as_float(raw[u >> 5][u & 31]),
+                                                     __uint_as_float(raw[(u + 1) >> 5][(u + 1) & 31]));
                         r = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                     } else {
                         float mn4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
@@ -425,16 +427,23 @@ fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
                 const float c = bias - ((m_ref == -INFINITY) ? 0.f : m_ref);   // P = 2^(S sc + c)
                 uint32_t pk[32];
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};     // 4 independent chains
+                // two keys per f32x2 instruction: the FMA and the running sums
+                const unsigned long long sc2 = f2_pack(sc, sc), c2 = f2_pack(c, c);
+                unsigned long long l2[4] = {0ull, 0ull, 0ull, 0ull};     // 4 independent chains of pairs
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int u = 2 * e;
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(raw[u >> 5][u & 31]), sc, c));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(raw[(u + 1) >> 5][(u + 1) & 31]), sc, c));
-                    l4[e & 3] += p0 + p1;
+                    const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[u >> 5][u & 31]),
+                                                              __uint_as_float(raw[(u + 1) >> 5][(u + 1) & 31])),
+                                                      sc2, c2));
+                    const float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
+                    l2[e & 3] = f2_add(l2[e & 3], f2_pack(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
                 }
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                {
+                    const float2 a0 = f2_unpack(f2_add(l2[0], l2[1])), a1 = f2_unpack(f2_add(l2[2], l2[3]));
+                    l += (a0.x + a0.y) + (a1.x + a1.y);
+                }
                 tmem_st32(tT + 64 * buf, pk);
                 if (rescale) {
                     // O is rescaled in TMEM: PV of the previous step must be complete

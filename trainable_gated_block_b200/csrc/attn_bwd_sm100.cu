@@ -88,7 +88,7 @@ struct Params {
 // where off = log2 g - lse (log2 units) or -inf for a dead row; keys above
 // `lim` are masked (the diagonal block, kMask). dS' (dS times sm_scale) is
 // rounded to bf16 into the row's 128-byte-swizzled tile, and P too when a P
-// tile is given. Returns the row's sum of dS'.
+// tile is given (the dq kernel gives none). Returns the row's sum of dS'.
 template <bool kMask>
 __device__ __forceinline__ float pds_half(const uint32_t (&sv)[32], const uint32_t (&pv)[32], int hf, float scale2,
                                           float off, float sm_scale, float drs, int lim, uint8_t* bufP,
@@ -527,13 +527,14 @@ constexpr uint32_t kSmem = kOffBar + 1024 + 1024;
 constexpr uint32_t kTmAccV = 256, kTmAccK = 320;
 
 // warps: 0 TMA; 2-5 / 6-9 softmax warpgroups 0 / 1 (both on every step, keys
-// [32 w, 32 w + 32)); issuing warps 1: S = Q K^T, 10: dP = dO V^T,
-// 11: dV^T += dO^T P, 12: dK^T += Q^T dS
+// [32 w, 32 w + 32); each writes P, then dS); issuing warps 1: S = Q K^T,
+// 10: dP = dO V^T, 11: dV^T += dO^T P (as soon as P is written, so the dO
+// slot is released while dS is computed), 12: dK^T += Q^T dS
 
 struct Bars {
     uint64_t kv_full, kv_empty;
     uint64_t q_full[kSlots], o_full[kSlots], slot_empty[kSlots];
-    uint64_t s_full[2], tm_free[2], pds_full, pds_empty;
+    uint64_t s_full[2], tm_free[2], pds_full, pds_empty, p_full, p_empty;
     uint64_t acc_full, acc_empty;
     uint64_t drain[4];
     uint32_t tmem_base;
@@ -628,8 +629,10 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             mbar_init(&bars->s_full[b], 2);
             mbar_init(&bars->tm_free[b], 256);
         }
-        mbar_init(&bars->pds_full, 256);
-        mbar_init(&bars->pds_empty, 2);
+        mbar_init(&bars->pds_full, 256);                // dS written
+        mbar_init(&bars->pds_empty, 1);                 // dS read (the dK^T warp)
+        mbar_init(&bars->p_full, 256);                  // P written
+        mbar_init(&bars->p_empty, 1);                   // P read (the dV^T warp)
         mbar_init(&bars->acc_full, 2);
         mbar_init(&bars->acc_empty, 256);
         for (int w = 0; w < 4; ++w) mbar_init(&bars->drain[w], 1);
@@ -756,7 +759,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (!(ok = mbar_wait_warp(&bars->acc_empty, (item_it & 1) ^ 1, abort, p.status))) break;
                 ++item_it;
                 for (int m = 0; m < N && ok; ++m, ++g) {
-                    if (!(ok = mbar_wait_warp(&bars->pds_full, g & 1, abort, p.status))) break;
+                    if (!(ok = mbar_wait_warp(is_v ? &bars->p_full : &bars->pds_full, g & 1, abort, p.status))) break;
                     tc_fence_after();
                     const int sl = (2 * g + (is_v ? 1 : 0)) % kSlots;
                     const uint32_t at_lo = sdesc_lo(s_base + kOffRing + sl * kTile, kTileAtom);   // MN-major
@@ -765,7 +768,7 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                         mma_ss_e(acc, at_lo + ((kk * 2048) >> 4), kHi, pb_lo + ((kk * 2048) >> 4), kHi, id_t,
                                  (m > 0 || kk > 0) ? 1u : 0u);
                     mma_commit_e(&bars->slot_empty[sl]);   // the tile's last reader
-                    mma_commit_e(&bars->pds_empty);
+                    mma_commit_e(is_v ? &bars->p_empty : &bars->pds_empty);
                 }
                 if (!ok) break;
                 mma_commit_e(&bars->acc_full);
@@ -812,12 +815,54 @@ dkv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bars->tm_free[buf]);       // S/dP columns may be refilled
-                // the accumulation MMAs of the previous step have read the P / dS tiles
+                // P first, so that dV^T += dO^T P (and the release of the dO slot) starts
+                // while dS is computed; each tile is rewritten once its MMA of the
+                // previous step has read it
+                unsigned long long pr[16];              // P of the half's keys, in pairs
+                if (g > 0 && !(ok = mbar_wait(&bars->p_empty, (g - 1) & 1, abort, p.status))) break;
+                {
+                    const unsigned long long sc2 = f2_pack(p.scale2, p.scale2), off2 = f2_pack(off, off);
+                    const int lim = sm.cur ? r_in : 63;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pp[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int e = 8 * c + 2 * e2;
+                            float2 x = f2_unpack(
+                                f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, off2));
+                            if (sm.cur) {
+                                x.x = (32 * w + e > lim) ? -INFINITY : x.x;
+                                x.y = (32 * w + e + 1 > lim) ? -INFINITY : x.y;
+                            }
+                            const float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
+                            pr[4 * c + e2] = f2_pack(p0, p1);
+                            pp[e2] = pack_bf16x2(p0, p1);
+                        }
+                        *reinterpret_cast<uint4*>(bufP + sw128_offset(row, 4 * w + c)) =
+                            make_uint4(pp[0], pp[1], pp[2], pp[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&bars->p_full);
                 if (g > 0 && !(ok = mbar_wait(&bars->pds_empty, (g - 1) & 1, abort, p.status))) break;
-                if (sm.cur)                             // causal mask on the diagonal block
-                    pds_half<true>(sv, pv, w, p.scale2, off, p.sm_scale, drs, r_in, bufP, bufS, row);
-                else
-                    pds_half<false>(sv, pv, w, p.scale2, off, p.sm_scale, drs, 63, bufP, bufS, row);
+                {
+                    const unsigned long long sm2 = f2_pack(p.sm_scale, p.sm_scale), nd2 = f2_pack(-drs, -drs);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t dd[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int e = 8 * c + 2 * e2;
+                            const unsigned long long dp =
+                                f2_fma(f2_pack(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])), sm2, nd2);
+                            const float2 d = f2_unpack(f2_mul(pr[4 * c + e2], dp));
+                            dd[e2] = pack_bf16x2(d.x, d.y);
+                        }
+                        *reinterpret_cast<uint4*>(bufS + sw128_offset(row, 4 * w + c)) =
+                            make_uint4(dd[0], dd[1], dd[2], dd[3]);
+                    }
+                }
                 fence_proxy_async_smem();
                 mbar_arrive(&bars->pds_full);
             }

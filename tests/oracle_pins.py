@@ -656,10 +656,25 @@ def pin_standin_scores_decode(O):
                                                                       atol=1e-13)
 
 
+def pin_attended_tiles(O):
+    """The attended-tile count the throughput is quoted on, by brute force: every
+    query head of every query block attends its own block and each kept one."""
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, NQB, K = 2, 6, 2, 10, 3
+    s = rng.standard_normal((B, Hkv, NQB, NQB))
+    _, cnt, _, _ = O.select(s, K, O.prefill_history(NQB))
+    brute = 0
+    for b in range(B):
+        for hq in range(Hq):
+            for i in range(NQB):
+                brute += 1 + min(K, i)          # own block + min(K, #history) kept ones
+    assert O.attended_tiles(cnt, Hq, Hkv) == brute == B * Hq * (1 + 2 + 3 + 4 * 7)
+
+
 ALL_PINS = [
     pin_topk_rank, pin_select_gates, pin_golden, pin_dense_equivalence, pin_block_diagonal,
     pin_general_sdpa, pin_bruteforce_loops, pin_finite_differences, pin_shift_invariance,
     pin_sparsity, pin_probabilities, pin_decode_vs_sdpa, pin_decode_vs_prefill, pin_standin_scores,
     pin_partial_block_sdpa, pin_partial_block_prefix, pin_varlen_sdpa, pin_varlen_finite_differences,
-    pin_standin_scores_decode,
+    pin_standin_scores_decode, pin_attended_tiles,
 ]

@@ -77,6 +77,8 @@ MUTANTS = {
                                                 "nh = int((kv_len[n] + BLOCK - 1) // BLOCK)\n        for h in range(Hkv):\n            qm"),
     "standin_transposed": ("s[b, h] = (qp[b, :, h, :] @ kp[b, :, h, :].T) / math.sqrt(D)",
                            "s[b, h] = (kp[b, :, h, :] @ qp[b, :, h, :].T) / math.sqrt(D)"),
+    "attended_tiles_without_current_block": ("return int((cnt + 1).sum()) * (Hq // Hkv)",
+                                             "return int(cnt.sum()) * (Hq // Hkv)"),
 }
 
 

@@ -279,6 +279,7 @@ sas_status sas_pool_pages(const void *k_cache, int num_pages, int Hkv, int D, in
  * s          device fp32 [N, Hkv, ld_s] (output; entries j < nh written),
  *            ld_s >= the longest history (<= 16384 blocks).
  * idx, cnt, log_gate, lse_s   device [N, Hkv, K], [N, Hkv], [N, Hkv, K], [N, Hkv].
+ * SAS_ERR_UNSUPPORTED for N * Hkv > 65535.
  */
 sas_status sas_score_select_decode(const void *q, const float *kpool, int num_pages,
                                    const int32_t *page_table, int max_pages, const int32_t *kv_len,

@@ -146,3 +146,35 @@ def test_score_select_rejects_bad_arguments(L):
     assert f(*bad) == sas.SAS_ERR_INVALID_ARG
     bad = list(args); bad[18] = 16                          # workspace too small
     assert f(*bad) == sas.SAS_ERR_INVALID_ARG
+
+
+def test_pool_pages_and_decode_scorer_reject_bad_arguments(L):
+    pool = L.sas_pool_pages
+    #          k_cache pages Hkv D   psz pages n   kpool stream
+    args = [FAKE, 4, 2, 128, 64, None, 0, FAKE, None]
+    bad = list(args); bad[0] = None
+    assert pool(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[4] = 32                            # page size
+    assert pool(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[3] = 96                            # D
+    assert pool(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[7] = ctypes.c_void_p(0x10004)     # kpool alignment
+    assert pool(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[5] = FAKE; bad[6] = 0             # an empty page list is a no-op
+    assert pool(*bad) == sas.SAS_OK
+
+    dec = L.sas_score_select_decode
+    #       q     kpool pages ptab max  kv_len N  Hq Hkv D    psz noise ld_n K  s     ld_s idx   cnt   lg    lse   stream
+    args = [FAKE, FAKE, 8, FAKE, 4, FAKE, 2, 8, 2, 128, 64, None, 0, 2, FAKE, 4, FAKE, FAKE, FAKE, FAKE, None]
+    bad = list(args); bad[3] = None                          # no page table
+    assert dec(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[7] = 6; bad[8] = 4                 # Hq % Hkv
+    assert dec(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[11] = FAKE; bad[12] = 3            # noise rows shorter than ld_s
+    assert dec(*bad) == sas.SAS_ERR_INVALID_ARG
+    bad = list(args); bad[15] = 16385                        # rows longer than the selection handles
+    assert dec(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[6] = 40000                         # N * Hkv above a grid dimension
+    assert dec(*bad) == sas.SAS_ERR_UNSUPPORTED
+    bad = list(args); bad[1] = ctypes.c_void_p(0x10004)     # kpool alignment
+    assert dec(*bad) == sas.SAS_ERR_INVALID_ARG

@@ -373,6 +373,8 @@ sas_status sas_score_select_decode(const void* q, const float* kpool, int num_pa
     if (D != 64 && D != 128) return fail(SAS_ERR_UNSUPPORTED, "%s: D=%d (only 64 or 128)", fn, D);
     if (noise && ld_noise < ld_s) return fail(SAS_ERR_INVALID_ARG, "%s: ld_noise=%d < ld_s=%d", fn, ld_noise, ld_s);
     if (ld_s > kMaxHistory) return fail(SAS_ERR_UNSUPPORTED, "%s: rows of more than %d history blocks", fn, kMaxHistory);
+    if ((long long)N * Hkv > 65535)     // grid dimension of the scoring kernel
+        return fail(SAS_ERR_UNSUPPORTED, "%s: N*Hkv=%lld above 65535", fn, (long long)N * Hkv);
     if (!aligned16(kpool)) return fail(SAS_ERR_INVALID_ARG, "%s: kpool not 16-byte aligned", fn);
     int* st = status_ptr();
     if (!st) return fail(SAS_ERR_CUDA, "%s: no CUDA device", fn);

@@ -114,6 +114,17 @@ def prefill_tiles(cfg):
     return per_head * cfg.B * cfg.Hq
 
 
+def prefill_causal_flops(cfg):
+    """The causal-exact count: 14 D flops per (query, key) pair actually attended,
+    64 x rows for a kept history block and the causal triangle rows (rows + 1) / 2
+    for the query block's own block (rows = 64, or fewer for a partial last block)."""
+    per_head = 0
+    for i in range(cfg.NQB):
+        rows = min(BLOCK, cfg.S - i * BLOCK)
+        per_head += min(cfg.K, i) * BLOCK * rows + rows * (rows + 1) // 2
+    return 14 * cfg.D * per_head * cfg.B * cfg.Hq
+
+
 def decode_bytes(cfg, kv_len, cnt):
     """Algorithmic HBM bytes of one decode call: kept K/V pages (full history
     pages, the current block's valid tokens), q, o, selection and page ids."""
@@ -357,11 +368,13 @@ def run_ours(a):
             "metric": "SAS gated block-sparse attn fwd+bwd TFLOPS & decode HBM GB/s vs roofline",
             "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "value_causal_exact": round(weak_tflops(world, prefill_causal_flops(pc), prefill_ms), 3),
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) q/k/v/dO, pooled stand-in scores)",
             "config": {
                 "workload": f"{pc.name} select+fwd+bwd, then {dc.name} select+paged decode",
                 "prefill": dict(B=pc.B, S=pc.S, Hq=pc.Hq, Hkv=pc.Hkv, D=pc.D, K=pc.K, block=BLOCK,
-                                attended_tiles=tiles, flops_per_step=flops_fb),
+                                attended_tiles=tiles, flops_per_step=flops_fb,
+                                flops_per_step_causal_exact=prefill_causal_flops(pc)),
                 "decode": dict(N=dc.N, Hq=dc.Hq, Hkv=dc.Hkv, D=dc.D, K=dc.K, ctx="8k..64k",
                                algorithmic_bytes=dec_bytes),
                 "l2": "inputs larger than L2 (prefill q/k/v/o/dO about 0.9 GB, decode pages 0.54 GB per step)",

@@ -103,3 +103,17 @@ def test_dkv_balance_model():
     assert r["items"] == 4 and r["steps_max_item"] == 4
     assert r["cta_steps_max"] == 5 and r["cta_steps_mean"] == 4.0
     assert r["cta_max_over_mean"] == 1.25
+
+
+@pytest.mark.parametrize("name,gflop", [
+    ("qwen3-8b-32k", 3785.3),       # the causal-exact counts of the scope table
+    ("qwen3-4b-8k", 464.4),
+    ("qwen3-14b-2x32k", 2536.7),
+])
+def test_prefill_causal_flops(name, gflop):
+    cfg = inputs.workload(name)
+    assert abs(bench.prefill_causal_flops(cfg) / 1e9 - gflop) < 0.06
+    # a partial last block: the tile count rounds it up, the causal count does not
+    small = inputs.PrefillConfig("p", "bf16", 1, 100, 2, 1, 128, 1, "normal", 1.0, seed=1)
+    pairs = (64 * 65 // 2) + (1 * 64 * 36 + 36 * 37 // 2)     # block 0; block 1 (36 rows, 1 kept block)
+    assert bench.prefill_causal_flops(small) == 14 * 128 * pairs * 2

@@ -310,7 +310,10 @@ size_t sas_decode_workspace_size(int N, int Hq, int Hkv, int D, int K);
  * idx, cnt, log_gate   device [N, Hkv, K], [N, Hkv], [N, Hkv, K] from
  *            sas_select (decode mode).
  * o          device bf16 [N, Hq, D] (output). lse: device fp32 [N, Hq] or NULL.
- * workspace  device, ws_bytes >= sas_decode_workspace_size(...).
+ * workspace  device, ws_bytes >= sas_decode_workspace_size(...), 256-byte
+ *            aligned; contents on entry do not matter.
+ * SAS_ERR_UNSUPPORTED unless D = 128, page_size = 64 and the GQA group size
+ * Hq/Hkv is 1, 2, 4, 5 or 8.
  */
 sas_status sas_decode_paged(const void *q, const void *k_cache, const void *v_cache,
                             int num_pages, const int32_t *page_table, int max_pages,
